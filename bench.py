@@ -1,0 +1,453 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged-attention hot path on B200.
+
+One step = one pass of the whole hot path over one batch: pa_kv_write of the
+step's new K/V rows, then pa_attention_mixed (plan, decode, split-KV reduce,
+prefill as the batch needs).  The headline workload is the Llama-3-8B-shaped
+decode batch (256 requests, context U[512, 4096], 32 q / 8 kv heads, head_dim
+128, 70k-block pool); the metric is KV bytes the attention must read per
+second (sum over requests of seq_len * Hkv * D * 2 tensors * 2 bytes, exact
+tokens).  The mixed 8192-token step (192 decodes + prefill chunks) is timed
+too and reported as tokens/s under "mixed_step".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): replicas only -- every rank runs its own copy of the
+workload on its own GPU, no collective on the data path; the step time is the
+max over ranks (weak scaling).  --impl reference times the fp64 CPU oracle on
+a bounded sample of the same workload (the only reference this method has).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode paged-attn KV GB/s (% of HBM peak); mixed-step tokens/s on 1 B200"
+HEADLINE = "llama3_8b_decode"
+MIXED = "mixed_step_8192"
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def _kernel_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "paged_kv_cache_461_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(name, files):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel is unchanged since."""
+    p = os.path.join(PROFILES, f"{name}.json")
+    if not os.path.exists(p):
+        return None, None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != _kernel_hash(files):
+        return None, d
+    return d.get("dram_bytes_per_launch"), d
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, period_ms: int = 20):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 7:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+
+def _dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- our arm
+
+class Step:
+    """Device-resident inputs of one workload and the hot-path call sequence."""
+
+    def __init__(self, name: str, seed=None):
+        import torch
+
+        from paged_kv_cache_461_b200 import api
+        from paged_kv_cache_461_b200 import workloads as W
+        self.api = api
+        self.lay = W.workload_layout(name, seed)
+        self.vals = W.make_values_torch(self.lay, "cuda")
+        lay = self.lay
+        d = "cuda"
+        self.qsl = torch.from_numpy(lay.query_start_loc).to(d)
+        self.seq_lens = torch.from_numpy(lay.seq_lens).to(d)
+        self.bt = torch.from_numpy(lay.block_table).to(d)
+        self.slots = torch.from_numpy(lay.slot_mapping).to(d)
+        self.out = torch.empty_like(self.vals.q)
+        self.ws = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, self.vals.k_cache, lay.max_seq_len)
+        self.scale = 1.0 / math.sqrt(lay.head_dim)
+        G = lay.num_q_heads // lay.num_kv_heads
+        NT = 1 if G <= 8 else (2 if G <= 16 else 0)
+        cap = 8 * NT
+        max_splits = math.ceil(max(lay.max_seq_len, 1) / 1024) if NT else 0
+        self.launches_per_step = 2 + (1 if NT else 0) + (1 if NT and max_splits > 1 else 0) + \
+            (1 if lay.max_query_len * G > cap else 0)
+        self.kv_bytes = lay.kv_bytes()
+        q = lay.q_lens.astype(np.int64)
+        c = lay.ctx_lens.astype(np.int64)
+        pf = q * lay.num_q_heads // lay.num_kv_heads > cap
+        # causal (query, key) pairs of prefill rows: sum_i (c + i + 1)
+        pairs = (q * c + q * (q + 1) // 2)[pf].sum()
+        self.prefill_flops = float(pairs) * 4 * lay.num_q_heads * lay.head_dim
+        self.prefill_requests = np.nonzero(pf)[0]
+
+    def kv_write(self):
+        v = self.vals
+        self.api.kv_write(v.k_new, v.v_new, self.slots, v.k_cache, v.v_cache)
+
+    def attention(self):
+        lay, v = self.lay, self.vals
+        self.api.attention_mixed(v.q, v.k_cache, v.v_cache, self.qsl, self.seq_lens, self.bt, lay.max_query_len,
+                                 lay.max_seq_len, softmax_scale=self.scale, out=self.out, workspace=self.ws)
+
+    def step(self):
+        self.kv_write()
+        self.attention()
+
+
+def _time_region(fn, steps, warmup, ws, sub_events=None):
+    """W untimed steps, then EXACTLY `steps` steps between barrier+sync on both sides."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    stream = torch.cuda.current_stream()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        fn()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    return t0.elapsed_time(t1)
+
+
+def _attention_only_ms(st: Step, steps: int):
+    """Average duration of the attention launches inside a step loop (events on the launching stream)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    evs = []
+    for _ in range(steps):
+        st.kv_write()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        st.attention()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def _prefill_only(st: Step, steps: int, warmup: int):
+    """Time pa_attention_mixed on the prefill chunks of the mixed step alone."""
+    import torch
+    from paged_kv_cache_461_b200 import workloads as W
+    lay = st.lay
+    idx = st.prefill_requests
+    qsl = lay.query_start_loc
+    rows = np.concatenate([np.arange(qsl[r], qsl[r + 1]) for r in idx])
+    sub = W.StepLayout("prefill_only", lay.num_q_heads, lay.num_kv_heads, lay.head_dim, lay.num_blocks,
+                       lay.q_lens[idx], lay.ctx_lens[idx], lay.block_table[idx])
+    q = st.vals.q[torch.from_numpy(rows).cuda()].contiguous()
+    qsl_d = torch.from_numpy(sub.query_start_loc).cuda()
+    sl_d = torch.from_numpy(sub.seq_lens).cuda()
+    bt_d = torch.from_numpy(sub.block_table).cuda()
+    out = torch.empty_like(q)
+    ws = st.api.alloc_workspace(sub.num_seqs, sub.num_tokens, sub.num_q_heads, st.vals.k_cache, sub.max_seq_len)
+
+    def call():
+        st.api.attention_mixed(q, st.vals.k_cache, st.vals.v_cache, qsl_d, sl_d, bt_d, sub.max_query_len,
+                               sub.max_seq_len, softmax_scale=st.scale, out=out, workspace=ws)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def _e2e(st: Step, steps: int, warmup: int):
+    """Same metric through the public API with host buffers: pinned H2D of the step's inputs, the two
+    C-ABI calls, D2H of the output, all inside the timed region."""
+    import torch
+    v = st.vals
+    host = {k: t.cpu().pin_memory() for k, t in
+            (("q", v.q), ("k_new", v.k_new), ("v_new", v.v_new), ("slots", st.slots), ("qsl", st.qsl),
+             ("seq_lens", st.seq_lens), ("bt", st.bt))}
+    dev = {k: torch.empty_like(t, device="cuda") for k, t in host.items()}
+    out_h = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    lay = st.lay
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def one():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        st.api.kv_write(dev["k_new"], dev["v_new"], dev["slots"], v.k_cache, v.v_cache)
+        st.api.attention_mixed(dev["q"], v.k_cache, v.v_cache, dev["qsl"], dev["seq_lens"], dev["bt"],
+                               lay.max_query_len, lay.max_seq_len, softmax_scale=st.scale, out=st.out,
+                               workspace=st.ws)
+        out_h.copy_(st.out, non_blocking=True)
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return ms, h2d, d2h
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+
+def _oracle_sample(name: str, n_requests: int, seed=None):
+    """A bounded sample of the workload (first n requests) as host arrays for the oracle."""
+    from paged_kv_cache_461_b200 import workloads as W
+    lay = W.workload_layout(name, seed)
+    idx = np.arange(min(n_requests, lay.num_seqs))
+    sub = W.build_layout(name + "_sample", lay.ctx_lens[idx], lay.q_lens[idx], num_q_heads=lay.num_q_heads,
+                         num_kv_heads=lay.num_kv_heads, head_dim=lay.head_dim, seed=lay.seed)
+    vals = W.make_values_numpy(sub)
+    return sub, vals
+
+
+def cpu_oracle_run(name: str, target_s: float = 15.0, seed=None):
+    """Time the oracle (as it stands) on a request sample sized for about target_s of CPU work."""
+    import oracle
+    from paged_kv_cache_461_b200 import workloads as W
+    full = W.workload_layout(name, seed).num_seqs
+
+    def run(n):
+        sub, vals = _oracle_sample(name, n, seed)
+        kc, vc = oracle.kv_write(vals.k_new, vals.v_new, sub.slot_mapping, vals.k_cache, vals.v_cache)
+        t0 = time.perf_counter()
+        oracle.attention_for(sub, kc, vc, vals.q)
+        return sub, time.perf_counter() - t0
+
+    sub, dt = run(min(8, full))
+    n = int(min(full, max(sub.num_seqs, sub.num_seqs * target_s / max(dt, 1e-3))))
+    if n > sub.num_seqs:
+        sub, dt = run(n)
+    cores = oracle.num_cores()
+    return {"value": sub.kv_bytes() / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {sub.num_seqs} of the {full} requests of {name} "
+                      f"({sub.kv_bytes() / 1e9:.3f} GB of KV, {dt:.2f} s, fp64, {cores} threads)"}
+
+
+def reference_arm(args, ws, rank):
+    if rank != 0:
+        return
+    import oracle
+    t_steps = []
+    sub, vals = _oracle_sample(HEADLINE, 8)
+    kc, vc = oracle.kv_write(vals.k_new, vals.v_new, sub.slot_mapping, vals.k_cache, vals.v_cache)
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.attention_for(sub, kc, vc, vals.q)
+        t_steps.append(time.perf_counter() - t0)
+        if sum(t_steps) > 120:
+            break
+    dt = statistics.mean(t_steps)
+    v = sub.kv_bytes() / dt / 1e9
+    cores = oracle.num_cores()
+    line = {"metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus, "steps": len(t_steps),
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": HEADLINE, "sample_requests": sub.num_seqs},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"first {sub.num_seqs} requests of {HEADLINE}, each step one oracle pass"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="headline only (no mixed step, e2e, prefill)")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    if args.impl == "reference":
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        reference_arm(args, ws, rank)
+        return
+
+    import torch
+    ws, rank, local = _dist_init()
+    torch.cuda.set_device(local)
+    from paged_kv_cache_461_b200 import build
+    if rank == 0 or ws == 1:
+        build.build()
+    _barrier(ws)
+    peaks = _peaks()
+
+    st = Step(args.workload)
+    sampler = ClockSampler(local)
+    ms_total = _time_region(st.step, args.steps, args.warmup, ws)
+    clocks = sampler.stop()
+    ms_total = _max_over_ranks(ms_total, ws)
+    ms_step = ms_total / args.steps
+    value = ws * st.kv_bytes / (ms_step * 1e-3) / 1e9
+
+    # dominant kernel roofline: the attention launches (plan + decode + reduce), events on their stream
+    att_ms = _attention_only_ms(st, max(20, min(args.steps, 200)))
+    achieved = st.kv_bytes / (att_ms * 1e-3) / 1e9
+    traffic, _ = _traffic("decode_llama3_8b_decode", ["decode.cu", "ptx.cuh", "pa_internal.cuh"])
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "kernel": "pa_attention_mixed (plan + decode_kernel + reduce_kernel)",
+                "algorithmic_bytes_per_launch": st.kv_bytes, "ms_per_launch": att_ms,
+                "peak_source": f"{peaks['source']} hbm_gbs (burst copy)"}
+
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**st.lay.describe(), "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                       "l2": f"inputs larger than L2 ({st.kv_bytes / 1e9:.2f} GB KV read per step), no flush",
+                       "step": "pa_kv_write + pa_attention_mixed"},
+            "roofline": roofline, "gpu_launches": st.launches_per_step * args.steps, "clocks": clocks}
+
+    if not args.no_extras and rank == 0:
+        e_ms, h2d, d2h = _e2e(st, max(10, min(args.steps, 100)), args.warmup)
+        line["e2e"] = {"value": st.kv_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    if not args.no_extras:
+        del st
+        torch.cuda.empty_cache()
+        mx = Step(MIXED)
+        mk = max(10, min(args.steps, 100))
+        m_ms = _max_over_ranks(_time_region(mx.step, mk, args.warmup, ws), ws) / mk
+        pf_ms = _prefill_only(mx, mk, args.warmup)
+        pf_tf = mx.prefill_flops / (pf_ms * 1e-3) / 1e12
+        line["mixed_step"] = {
+            "value": ws * mx.lay.num_tokens / (m_ms * 1e-3), "unit": "tokens/s", "ms_per_step": m_ms,
+            "workload": mx.lay.describe(), "kv_bytes_per_step": mx.kv_bytes,
+            "prefill_flops_per_step": mx.prefill_flops,
+            "prefill_roofline": {"bound": "tensor", "achieved": pf_tf, "peak": peaks["bf16_tflops"],
+                                 "unit": "TFLOP/s", "frac": pf_tf / peaks["bf16_tflops"], "ms_per_launch": pf_ms,
+                                 "kernel": "pa_attention_mixed on the prefill chunks alone (prefill_kernel)",
+                                 "peak_source": f"{peaks['source']} bf16_tflops (burst)"}}
+        line["gpu_launches"] += mx.launches_per_step * mk
+
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_run(HEADLINE)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+/*
+ * pa.h -- C ABI of libpa_b200.so: paged attention over a block-managed KV
+ * cache for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow vLLM V1 as described in "Inside vLLM: Anatomy of a
+ * High-Throughput LLM Inference System" (restated on hn.213312.xyz and
+ * shengyayun.com):
+ *   - the KV cache is a pool of fixed 16-token blocks handed out and taken back
+ *     on demand, 16 tokens per block by default (hn.213312.xyz section 一,
+ *     scheduler paragraph; shengyayun.com, 关键实现细节 1);
+ *   - before the forward pass the runner copies metadata to the GPU and builds
+ *     positions and the slot mapping; the forward pass then runs a custom
+ *     paged-attention kernel over all sequences flattened into one
+ *     "super-sequence" (hn.213312.xyz section 一, forward-pass paragraph);
+ *   - one V1 step mixes prefill chunks and decode tokens (hn.213312.xyz
+ *     section 一 "调度器"; shengyayun.com 适用场景); a chunk attends to its
+ *     request's cached context and must give the same result as an unchunked
+ *     prefill (hn.213312.xyz section 二.1); prefix-cache hits reuse cached
+ *     blocks directly, so several block tables may name the same physical
+ *     blocks (section 二.2; shengyayun.com 关键实现细节 2).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; only the
+ *     pa_cache_desc_t / pa_attn_options_t structs are read from host memory,
+ *     during the call.  The library never allocates, frees or synchronises:
+ *     work is enqueued on `stream` and the call returns at once.
+ *   - bf16 tensors are IEEE bfloat16 (2 bytes per element).
+ *   - Host-side validation happens before anything is enqueued; a non-PA_OK
+ *     status means nothing was enqueued, except PA_ERR_CUDA (a launch failed).
+ *   - Metadata that lives on the device (seq_lens, block ids, slots) cannot be
+ *     validated on the host.  The kernels never read or write outside the
+ *     buffers described by the host-side sizes: a request whose lengths are
+ *     inconsistent is skipped and a block id outside the pool reads zeros;
+ *     both set a bit in the device status word (see pa_attention_mixed).
+ */
+#ifndef PA_B200_H
+#define PA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(PA_BUILD) && defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the same handle type); NULL is the legacy default stream. */
+typedef struct CUstream_st *pa_stream_t;
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,          /* null pointer, negative size, inconsistent shapes, aliasing */
+    PA_ERR_UNSUPPORTED = 2,          /* valid but not implemented: head_dim, block_size, GQA ratio, alignment */
+    PA_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace_bytes < pa_workspace_size_ex(...) */
+    PA_ERR_CUDA = 4                  /* a CUDA launch or driver call failed */
+} pa_status_t;
+
+/* Both caches have the layout [num_blocks][num_kv_heads][block_size][head_dim]
+ * bf16, contiguous: one (block, kv head) is block_size*head_dim*2 bytes
+ * (4 KiB at head_dim 128), the unit the kernels fetch.  Slot s is token
+ * s % block_size of block s / block_size. */
+typedef struct pa_cache_desc {
+    int64_t num_blocks;    /* > 0; num_blocks*num_kv_heads*block_size must be < 2^31 */
+    int32_t num_kv_heads;  /* > 0 */
+    int32_t head_dim;      /* 64 or 128 */
+    int32_t block_size;    /* 16 (vLLM's default block size) */
+} pa_cache_desc_t;
+
+/* Optional knobs of pa_attention_mixed_ex / pa_workspace_size_ex.  A NULL
+ * options pointer, or a zero field, takes the default. */
+typedef struct pa_attn_options {
+    int32_t kv_split_tokens; /* keys per split-KV partition of a decode request;
+                                0 = default (1024); else a positive multiple of 16 */
+    int32_t reserved[7];     /* must be zero */
+} pa_attn_options_t;
+
+/* Bits of the device status word (uint32 at byte 0 of the workspace). */
+#define PA_DEVICE_BAD_SEQ 1u      /* a request had q_len < 0, seq_len < q_len, seq_len > max_seq_len or
+                                     query rows outside [0, num_tokens); it was skipped */
+#define PA_DEVICE_BAD_BLOCK 2u    /* a block id outside [0, num_blocks) was read (as zeros) */
+#define PA_DEVICE_WAIT_TIMEOUT 4u /* a kernel gave up waiting on a copy or a tensor-core result */
+
+PA_API int32_t pa_abi_version(void); /* 1 */
+PA_API const char *pa_status_string(pa_status_t status);
+
+/*
+ * pa_kv_write -- scatter this step's new K and V rows into their cache slots.
+ * (hn.213312.xyz section 一: the slot mapping is built while inputs are
+ * prepared, and the KV tensors are allocated and bound once at start-up.)
+ *
+ *   k_cache[s / bs][h][s % bs][:] = k_new row t, head h   (same for V)
+ * for every token t < num_tokens with s = slot_mapping[t] >= 0 and every
+ * h < num_kv_heads.
+ *
+ * k_new, v_new: bf16; token t's row starts at element t*new_row_stride and
+ *   holds num_kv_heads*head_dim contiguous elements ([T, Hkv, D] when
+ *   new_row_stride == Hkv*D; larger strides read rows out of a fused QKV).
+ * slot_mapping: int64 [num_tokens]; < 0 marks a padding token (skipped).  A
+ *   slot >= num_blocks*block_size is skipped too.  Two tokens with the same
+ *   non-negative slot in one call leave that slot undefined.
+ * The copy is bit-exact; no other cache byte is written.
+ */
+PA_API pa_status_t pa_kv_write(const void *k_new, const void *v_new, int64_t new_row_stride,
+                        const int64_t *slot_mapping, int32_t num_tokens, void *k_cache, void *v_cache,
+                        const pa_cache_desc_t *cache, pa_stream_t stream);
+
+/*
+ * pa_build_slot_mapping -- the slot of every token of the step.
+ * (hn.213312.xyz section 一, forward-pass paragraph: positions and the slot
+ * mapping are prepared on the way into the forward pass.)
+ * Token i of request r (row query_start_loc[r] + i) sits at position
+ * p = seq_lens[r] - q_len_r + i and gets
+ *   slot = block_table[r*bt_stride + p / 16] * 16 + p % 16.
+ * query_start_loc int32 [num_seqs+1] (non-decreasing, last <= num_tokens),
+ * seq_lens int32 [num_seqs], block_table int32 [num_seqs, bt_stride],
+ * slot_mapping int64 [num_tokens] out.  Rows of a request with
+ * seq_len < q_len, or whose block index would reach bt_stride, get -1.
+ * Rows not covered by any request are left untouched.
+ */
+PA_API pa_status_t pa_build_slot_mapping(const int32_t *query_start_loc, const int32_t *seq_lens,
+                                  const int32_t *block_table, int32_t bt_stride, int32_t num_seqs,
+                                  int32_t num_tokens, int64_t *slot_mapping, pa_stream_t stream);
+
+/*
+ * pa_workspace_size[_ex] -- bytes of device workspace pa_attention_mixed[_ex]
+ * needs for these host-side bounds (0 on invalid arguments).  The value only
+ * grows with each argument, so one workspace sized for the largest step of a
+ * run serves every smaller step.
+ */
+PA_API size_t pa_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads,
+                         const pa_cache_desc_t *cache, int32_t max_seq_len);
+PA_API size_t pa_workspace_size_ex(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads,
+                            const pa_cache_desc_t *cache, int32_t max_seq_len,
+                            const pa_attn_options_t *options);
+
+/*
+ * pa_attention_mixed[_ex] -- causal attention of one mixed prefill/decode
+ * step over the paged cache.
+ * (hn.213312.xyz section 一 forward-pass paragraph and sections 二.1/二.2;
+ *  shengyayun.com 适用场景: the V1 scheduler puts prefill and decode work in
+ *  the same step.)
+ *
+ * Request r owns query rows [query_start_loc[r], query_start_loc[r+1]) of q;
+ * q_len_r is their count, seq_lens[r] = L_r counts its tokens in the cache
+ * including this step's (pa_kv_write must already have run on this stream),
+ * and c_r = L_r - q_len_r tokens were cached before the step.  Row i of the
+ * request is at position p = c_r + i; query head h uses kv head
+ * h / (num_q_heads / num_kv_heads) and attends keys 0..p of its request:
+ *   out[row][h] = sum_j softmax_j(softmax_scale * q . K_j) V_j.
+ * Key j of request r lives at block block_table[r*bt_stride + j/16], row j%16.
+ * Requests may appear in any order and may share physical blocks.
+ *
+ * q: bf16 [num_tokens, num_q_heads, head_dim], 16-byte aligned.
+ * k_cache, v_cache: per `cache`, 16-byte aligned.
+ * query_start_loc: int32 [num_seqs+1]; seq_lens: int32 [num_seqs];
+ * block_table: int32 [num_seqs, bt_stride] with bt_stride >= ceil(max_seq_len/16);
+ *   entries past ceil(L_r/16) are never read.
+ * max_query_len, max_seq_len: host-side upper bounds of q_len_r and L_r.
+ * out: bf16 [num_tokens, num_q_heads, head_dim]; must not overlap q.  Rows
+ *   that belong to no request are not written.
+ * lse: fp32 [num_tokens, num_q_heads] natural-log log-sum-exp of the scaled
+ *   scores, or NULL.
+ * workspace: device memory of at least pa_workspace_size_ex(...) bytes,
+ *   16-byte aligned, used only while the enqueued work runs; calls that can
+ *   run concurrently need distinct workspaces.  Byte 0 holds the device status
+ *   word (PA_DEVICE_* bits), reset by every call and readable after it.
+ *
+ * Supported: head_dim 64 or 128, block_size 16, num_q_heads/num_kv_heads a
+ * divisor of 128.  Errors: INVALID_ARG (null pointer, negative size,
+ * num_q_heads % num_kv_heads != 0, bt_stride too small, out overlapping q,
+ * nonzero reserved option), UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA.
+ */
+PA_API pa_status_t pa_attention_mixed(const void *q, int32_t num_q_heads, const void *k_cache,
+                               const void *v_cache, const pa_cache_desc_t *cache,
+                               const int32_t *query_start_loc, const int32_t *seq_lens,
+                               const int32_t *block_table, int32_t bt_stride, int32_t num_seqs,
+                               int32_t num_tokens, int32_t max_query_len, int32_t max_seq_len,
+                               float softmax_scale, void *out, float *lse, void *workspace,
+                               size_t workspace_bytes, pa_stream_t stream);
+PA_API pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, const void *k_cache,
+                                  const void *v_cache, const pa_cache_desc_t *cache,
+                                  const int32_t *query_start_loc, const int32_t *seq_lens,
+                                  const int32_t *block_table, int32_t bt_stride, int32_t num_seqs,
+                                  int32_t num_tokens, int32_t max_query_len, int32_t max_seq_len,
+                                  float softmax_scale, void *out, float *lse, void *workspace,
+                                  size_t workspace_bytes, const pa_attn_options_t *options,
+                                  pa_stream_t stream);
+
+/*
+ * pa_merge_attn_states -- the split-KV reduce on its own.
+ * Given attention states of num_parts disjoint key sets for each (row, head):
+ * normalised outputs part_out fp32 [num_rows, num_heads, num_parts, head_dim]
+ * and log-sum-exps part_lse fp32 [num_rows, num_heads, num_parts] (natural
+ * log; -inf marks an empty part), write
+ *   LSE = ln sum_s exp(lse_s),  out = sum_s exp(lse_s - LSE) * o_s
+ * as bf16 out [num_rows, num_heads, head_dim] and, if lse_out is not NULL,
+ * fp32 lse_out [num_rows, num_heads].  parts_per_row (int32 [num_rows], may be
+ * NULL) limits row i to its first parts_per_row[i] parts.  A row whose parts
+ * are all empty gets out = 0, lse = -inf.  head_dim 64 or 128.
+ */
+PA_API pa_status_t pa_merge_attn_states(const float *part_out, const float *part_lse, const int32_t *parts_per_row,
+                                 int32_t num_rows, int32_t num_heads, int32_t num_parts, int32_t head_dim,
+                                 void *out, float *lse_out, pa_stream_t stream);
+
+/*
+ * pa_debug_gather_kv -- test helper: contiguous copy of one request's first
+ * seq_len tokens of a cache, following its block table row (device int32
+ * [ceil(seq_len/16)]).  out: bf16 [seq_len, num_kv_heads, head_dim].  A block
+ * id outside the pool gives zero rows.
+ */
+PA_API pa_status_t pa_debug_gather_kv(const void *cache_ptr, const pa_cache_desc_t *cache, const int32_t *bt_row,
+                               int32_t seq_len, void *out, pa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_B200_H */

@@ -1,0 +1,210 @@
+"""ctypes binding of libpa_b200.so -- argument marshalling only.
+
+Every function here has the name of a C entry point in include/pa.h minus the
+``pa_`` prefix, takes torch CUDA tensors, passes their data pointers and the
+current stream to the library, and raises PaError on a non-PA_OK status.
+All arithmetic runs in the library's CUDA kernels; there is no fallback: if
+the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa_b200.so")
+
+PA_OK = 0
+STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_WORKSPACE_TOO_SMALL",
+                4: "PA_ERR_CUDA"}
+DEVICE_BAD_SEQ = 1
+DEVICE_BAD_BLOCK = 2
+DEVICE_WAIT_TIMEOUT = 4
+
+# every symbol include/pa.h declares
+EXPORTED = ("pa_abi_version", "pa_status_string", "pa_kv_write", "pa_build_slot_mapping", "pa_workspace_size",
+            "pa_workspace_size_ex", "pa_attention_mixed", "pa_attention_mixed_ex", "pa_merge_attn_states",
+            "pa_debug_gather_kv")
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int64), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("block_size", ctypes.c_int32)]
+
+
+class AttnOptions(ctypes.Structure):
+    _fields_ = [("kv_split_tokens", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+
+
+_lib = None
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+
+def lib():
+    """Open libpa_b200.so (built in place by paged_kv_cache_461_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_461_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.pa_abi_version.restype = _i32
+        L.pa_status_string.restype = ctypes.c_char_p
+        L.pa_status_string.argtypes = [ctypes.c_int]
+        L.pa_kv_write.argtypes = [_vp, _vp, _i64, _vp, _i32, _vp, _vp, ctypes.POINTER(CacheDesc), _vp]
+        L.pa_build_slot_mapping.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp]
+        L.pa_workspace_size.argtypes = [_i32, _i32, _i32, ctypes.POINTER(CacheDesc), _i32]
+        L.pa_workspace_size.restype = _sz
+        L.pa_workspace_size_ex.argtypes = [_i32, _i32, _i32, ctypes.POINTER(CacheDesc), _i32,
+                                           ctypes.POINTER(AttnOptions)]
+        L.pa_workspace_size_ex.restype = _sz
+        attn = [_vp, _i32, _vp, _vp, ctypes.POINTER(CacheDesc), _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                ctypes.c_float, _vp, _vp, _vp, _sz]
+        L.pa_attention_mixed.argtypes = attn + [_vp]
+        L.pa_attention_mixed_ex.argtypes = attn + [ctypes.POINTER(AttnOptions), _vp]
+        L.pa_merge_attn_states.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
+        L.pa_debug_gather_kv.argtypes = [_vp, ctypes.POINTER(CacheDesc), _vp, _i32, _vp, _vp]
+        for name in ("pa_kv_write", "pa_build_slot_mapping", "pa_attention_mixed", "pa_attention_mixed_ex",
+                     "pa_merge_attn_states", "pa_debug_gather_kv"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != PA_OK:
+        raise PaError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def cache_desc(k_cache: torch.Tensor) -> CacheDesc:
+    NB, Hkv, bs, D = k_cache.shape
+    return CacheDesc(NB, Hkv, D, bs)
+
+
+def _opts(kv_split_tokens: int) -> Optional[AttnOptions]:
+    if not kv_split_tokens:
+        return None
+    o = AttnOptions()
+    o.kv_split_tokens = int(kv_split_tokens)
+    return o
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if t.dtype != dtype or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA {dtype} tensor (got {t.dtype} on {t.device})")
+
+
+# ---------------------------------------------------------------- entry points
+
+def abi_version() -> int:
+    return int(lib().pa_abi_version())
+
+
+def kv_write(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, k_cache: torch.Tensor,
+             v_cache: torch.Tensor, stream=None) -> None:
+    """pa_kv_write: k_new/v_new [T, Hkv, D] (rows may be strided), slot_mapping int64 [T]."""
+    _need(k_new, torch.bfloat16, "k_new")
+    _need(slot_mapping, torch.int64, "slot_mapping")
+    T = slot_mapping.shape[0]
+    row_stride = k_new.stride(0) if T else k_new.shape[-1] * k_new.shape[-2]
+    if k_new.stride(0) != v_new.stride(0) or k_new.stride(-1) != 1 or k_new.stride(-2) != k_new.shape[-1]:
+        raise ValueError("k_new and v_new need the same row stride and contiguous [Hkv, D] rows")
+    d = cache_desc(k_cache)
+    _check(lib().pa_kv_write(_ptr(k_new), _ptr(v_new), row_stride, _ptr(slot_mapping), T, _ptr(k_cache),
+                             _ptr(v_cache), ctypes.byref(d), _stream(stream)), "pa_kv_write")
+
+
+def build_slot_mapping(query_start_loc: torch.Tensor, seq_lens: torch.Tensor, block_table: torch.Tensor,
+                       num_tokens: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.full((num_tokens,), -1, dtype=torch.int64, device=query_start_loc.device)
+    _check(lib().pa_build_slot_mapping(_ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
+                                       block_table.stride(0), seq_lens.shape[0], num_tokens, _ptr(out),
+                                       _stream(stream)), "pa_build_slot_mapping")
+    return out
+
+
+def workspace_size(num_seqs: int, num_tokens: int, num_q_heads: int, k_cache_or_desc, max_seq_len: int,
+                   kv_split_tokens: int = 0) -> int:
+    d = k_cache_or_desc if isinstance(k_cache_or_desc, CacheDesc) else cache_desc(k_cache_or_desc)
+    o = _opts(kv_split_tokens)
+    return int(lib().pa_workspace_size_ex(num_seqs, num_tokens, num_q_heads, ctypes.byref(d), max_seq_len,
+                                          ctypes.byref(o) if o else None))
+
+
+def alloc_workspace(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens=0) -> torch.Tensor:
+    n = workspace_size(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens)
+    if n == 0:
+        raise PaError(1, "pa_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=k_cache.device)
+
+
+def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, query_start_loc: torch.Tensor,
+                    seq_lens: torch.Tensor, block_table: torch.Tensor, max_query_len: int, max_seq_len: int,
+                    softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                    lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    kv_split_tokens: int = 0, stream=None) -> torch.Tensor:
+    """pa_attention_mixed[_ex]: q [T, Hq, D] bf16 -> out [T, Hq, D] bf16 (lse [T, Hq] fp32 if given)."""
+    _need(q, torch.bfloat16, "q")
+    T, Hq, D = q.shape
+    R = seq_lens.shape[0]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens)
+    d = cache_desc(k_cache)
+    o = _opts(kv_split_tokens)
+    _check(lib().pa_attention_mixed_ex(_ptr(q), Hq, _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
+                                       _ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
+                                       block_table.stride(0), R, T, int(max_query_len), int(max_seq_len),
+                                       float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       ctypes.byref(o) if o else None, _stream(stream)), "pa_attention_mixed")
+    return out
+
+
+def merge_attn_states(part_out: torch.Tensor, part_lse: torch.Tensor, parts_per_row: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None, lse_out: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """pa_merge_attn_states: part_out fp32 [N, H, S, D], part_lse fp32 [N, H, S] -> bf16 [N, H, D]."""
+    N, H, S, D = part_out.shape
+    if out is None:
+        out = torch.empty((N, H, D), dtype=torch.bfloat16, device=part_out.device)
+    _check(lib().pa_merge_attn_states(_ptr(part_out), _ptr(part_lse), _ptr(parts_per_row), N, H, S, D, _ptr(out),
+                                      _ptr(lse_out), _stream(stream)), "pa_merge_attn_states")
+    return out
+
+
+def debug_gather_kv(cache: torch.Tensor, bt_row: torch.Tensor, seq_len: int, stream=None) -> torch.Tensor:
+    NB, Hkv, bs, D = cache.shape
+    out = torch.empty((seq_len, Hkv, D), dtype=cache.dtype, device=cache.device)
+    d = cache_desc(cache)
+    _check(lib().pa_debug_gather_kv(_ptr(cache), ctypes.byref(d), _ptr(bt_row), seq_len, _ptr(out),
+                                    _stream(stream)), "pa_debug_gather_kv")
+    return out
+
+
+def read_device_status(workspace: torch.Tensor) -> int:
+    """The PA_DEVICE_* bits the last call that used this workspace left (synchronises)."""
+    return int(workspace[:4].view(torch.int32).item()) & 0xFFFFFFFF

@@ -1,0 +1,138 @@
+// kv_write.cu -- the KV-cache write (scatter of this step's K/V rows into their
+// 16-token blocks through the slot mapping), the slot-mapping builder and the
+// debug gather.  All three are pure data movement, bound by HBM bandwidth:
+// each warp moves whole (token, head) rows with 16-byte vector accesses, so
+// every load and store is a full 32-byte sector run.
+//
+// Semantics follow the model-runner step restated on hn.213312.xyz (section 一,
+// "前向传播"): prepare-inputs builds positions and the slot mapping, then the
+// forward pass writes each layer's new K/V into the cache before attention.
+#include <type_traits>
+
+#include "pa_internal.cuh"
+
+namespace pa {
+namespace {
+
+// One warp per token; lanes stride over the token's Hkv*D/VEC vectors of K and V.
+template <int VEC>
+__global__ void __launch_bounds__(256) kv_write_kernel(const uint16_t *__restrict__ k_new,
+                                                       const uint16_t *__restrict__ v_new, int64_t row_stride,
+                                                       const int64_t *__restrict__ slots, int num_tokens,
+                                                       uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
+                                                       int64_t num_blocks, int Hkv, int D)
+{
+    using Vec = typename std::conditional<VEC == 8, uint4, uint16_t>::type;
+    const int lane = threadIdx.x & 31;
+    const int warps_per_cta = blockDim.x >> 5;
+    const int64_t n_slots = num_blocks * kBlockSize;
+    const int vec_per_row = D / VEC;
+    const int vec_per_tok = Hkv * vec_per_row;
+    for (int64_t t = (int64_t)blockIdx.x * warps_per_cta + (threadIdx.x >> 5); t < num_tokens;
+         t += (int64_t)gridDim.x * warps_per_cta) {
+        const int64_t slot = slots[t];
+        if (slot < 0 || slot >= n_slots)
+            continue; // padding token, or a slot outside the pool: nothing is written
+        const int64_t blk = slot / kBlockSize;
+        const int off = (int)(slot % kBlockSize);
+        const uint16_t *ks = k_new + t * row_stride;
+        const uint16_t *vs = v_new + t * row_stride;
+        for (int i = lane; i < vec_per_tok; i += 32) {
+            const int h = i / vec_per_row;
+            const int e = (i - h * vec_per_row) * VEC;
+            const int64_t dst = ((blk * Hkv + h) * kBlockSize + off) * (int64_t)D + e;
+            const Vec kv = *reinterpret_cast<const Vec *>(ks + (int64_t)h * D + e);
+            const Vec vv = *reinterpret_cast<const Vec *>(vs + (int64_t)h * D + e);
+            *reinterpret_cast<Vec *>(k_cache + dst) = kv;
+            *reinterpret_cast<Vec *>(v_cache + dst) = vv;
+        }
+    }
+}
+
+// One CTA per request; threads stride over its query rows.
+__global__ void slot_mapping_kernel(const int32_t *__restrict__ qsl, const int32_t *__restrict__ seq_lens,
+                                    const int32_t *__restrict__ bt, int bt_stride, int num_tokens,
+                                    int64_t *__restrict__ slots)
+{
+    const int r = blockIdx.x;
+    const int qs = qsl[r], qe = qsl[r + 1];
+    const int q_len = qe - qs;
+    const int L = seq_lens[r];
+    const int ctx = L - q_len;
+    if (qs < 0 || qe > num_tokens || q_len <= 0)
+        return;
+    for (int i = threadIdx.x; i < q_len; i += blockDim.x) {
+        const int64_t p = (int64_t)ctx + i;
+        int64_t s = -1;
+        if (ctx >= 0 && p / kBlockSize < bt_stride)
+            s = (int64_t)bt[(int64_t)r * bt_stride + p / kBlockSize] * kBlockSize + p % kBlockSize;
+        slots[qs + i] = s;
+    }
+}
+
+// One warp per token of the request: copy its Hkv rows into out[j].
+__global__ void gather_kernel(const uint16_t *__restrict__ cache, int64_t num_blocks, int Hkv, int D,
+                              const int32_t *__restrict__ bt_row, int seq_len, uint16_t *__restrict__ out)
+{
+    const int lane = threadIdx.x & 31;
+    const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (j >= seq_len)
+        return;
+    const int64_t blk = bt_row[j / kBlockSize];
+    const bool ok = blk >= 0 && blk < num_blocks;
+    const int off = j % kBlockSize;
+    const int n = Hkv * D;
+    for (int i = lane; i < n; i += 32) {
+        const int h = i / D, d = i - h * D;
+        uint16_t v = 0;
+        if (ok)
+            v = cache[((blk * Hkv + h) * kBlockSize + off) * (int64_t)D + d];
+        out[(int64_t)j * n + i] = v;
+    }
+}
+
+} // namespace
+
+cudaError_t launch_kv_write(const void *k_new, const void *v_new, int64_t row_stride, const int64_t *slots,
+                            int num_tokens, void *k_cache, void *v_cache, int64_t num_blocks, int Hkv, int D,
+                            cudaStream_t s)
+{
+    const bool vec_ok = ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new) |
+                          reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) % 16 == 0) &&
+                        (row_stride % 8 == 0) && (D % 8 == 0);
+    const int threads = 256;
+    const int warps = threads / 32;
+    int64_t blocks = ((int64_t)num_tokens + warps - 1) / warps;
+    if (blocks > 148 * 16)
+        blocks = 148 * 16;
+    if (blocks < 1)
+        blocks = 1;
+    if (vec_ok)
+        kv_write_kernel<8><<<(unsigned)blocks, threads, 0, s>>>(
+            static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new), row_stride, slots, num_tokens,
+            static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache), num_blocks, Hkv, D);
+    else
+        kv_write_kernel<1><<<(unsigned)blocks, threads, 0, s>>>(
+            static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new), row_stride, slots, num_tokens,
+            static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache), num_blocks, Hkv, D);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_slot_mapping(const int32_t *qsl, const int32_t *seq_lens, const int32_t *bt, int bt_stride,
+                                int num_seqs, int num_tokens, int64_t *slots, cudaStream_t s)
+{
+    slot_mapping_kernel<<<num_seqs, 128, 0, s>>>(qsl, seq_lens, bt, bt_stride, num_tokens, slots);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D, const int32_t *bt_row, int seq_len,
+                          void *out, cudaStream_t s)
+{
+    const int threads = 256;
+    const int blocks = (seq_len + 7) / 8;
+    gather_kernel<<<blocks, threads, 0, s>>>(static_cast<const uint16_t *>(cache), num_blocks, Hkv, D, bt_row,
+                                             seq_len, static_cast<uint16_t *>(out));
+    return cudaGetLastError();
+}
+
+} // namespace pa

@@ -1,0 +1,249 @@
+// plan_merge.cu -- device-side work decomposition of a mixed step, and the
+// split-KV reduce (merge of attention states over disjoint key ranges).
+//
+// Plan: one CTA reads query_start_loc / seq_lens, classifies each request as
+// decode (q_len * G small enough for the warp-MMA decode kernel) or prefill
+// (tensor-core tiles of 128 query rows), and writes the work lists the next
+// kernels index by blockIdx.  Nothing returns to the host, so the whole step
+// stays asynchronous and capturable in a CUDA graph.  The V1 scheduler puts
+// decodes first and prefill chunks after them (hn.213312.xyz section 一,
+// "调度器"), but nothing here depends on that order.
+//
+// Merge: for each (row, head) with parts s = 0..S-1 holding normalised
+// outputs o_s and natural-log LSEs, LSE = ln sum exp(lse_s) and
+// out = sum exp(lse_s - LSE) o_s -- the flash-decoding second pass, one warp
+// per (row, head), fp32 throughout, bf16 output.
+#include <math_constants.h>
+
+#include "pa_internal.cuh"
+
+namespace pa {
+namespace {
+
+__device__ __forceinline__ int warp_incl_scan(int v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o)
+            v += n;
+    }
+    return v;
+}
+
+// Exclusive scan of three counters across a 1024-thread CTA.
+__device__ __forceinline__ void cta_excl_scan3(int a, int b, int c, int &ea, int &eb, int &ec, int &ta, int &tb,
+                                               int &tc)
+{
+    __shared__ int sa[32], sb[32], sc[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ia = warp_incl_scan(a), ib = warp_incl_scan(b), ic = warp_incl_scan(c);
+    if (lane == 31) {
+        sa[warp] = ia;
+        sb[warp] = ib;
+        sc[warp] = ic;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        int xa = lane < nw ? sa[lane] : 0, xb = lane < nw ? sb[lane] : 0, xc = lane < nw ? sc[lane] : 0;
+        xa = warp_incl_scan(xa);
+        xb = warp_incl_scan(xb);
+        xc = warp_incl_scan(xc);
+        if (lane < nw) {
+            sa[lane] = xa;
+            sb[lane] = xb;
+            sc[lane] = xc;
+        }
+    }
+    __syncthreads();
+    const int wa = warp ? sa[warp - 1] : 0, wb = warp ? sb[warp - 1] : 0, wc = warp ? sc[warp - 1] : 0;
+    ea = wa + ia - a;
+    eb = wb + ib - b;
+    ec = wc + ic - c;
+    const int nw = blockDim.x >> 5;
+    ta = sa[nw - 1];
+    tb = sb[nw - 1];
+    tc = sc[nw - 1];
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p)
+{
+    WsHeader *hdr = p.hdr;
+    if (threadIdx.x == 0)
+        hdr->status = 0u;
+    int carry_dec = 0, carry_pf = 0, carry_red = 0;
+    for (int base = 0; base < p.num_seqs; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        int n_dec = 0, n_pf = 0, red = 0;
+        if (r < p.num_seqs) {
+            const int qs = p.qsl[r], qe = p.qsl[r + 1];
+            const int q_len = qe - qs;
+            const int L = p.seq_lens[r];
+            const bool bad = qs < 0 || qe > p.num_tokens || q_len < 0 || L < q_len || L > p.max_seq_len;
+            if (bad) {
+                atomicOr(&hdr->status, PA_DEVICE_BAD_SEQ);
+            } else if (q_len > 0) {
+                if (q_len * p.G <= p.dec_rows_cap) {
+                    n_dec = (L + p.split_tokens - 1) / p.split_tokens;
+                    red = n_dec > 1 ? 1 : 0;
+                } else {
+                    n_pf = (q_len * p.G + kPrefillRows - 1) / kPrefillRows;
+                }
+            }
+        }
+        int ed, ep, er, td, tp, tr;
+        cta_excl_scan3(n_dec, n_pf, red, ed, ep, er, td, tp, tr);
+        for (int s = 0; s < n_dec; ++s)
+            p.dec_units[carry_dec + ed + s] = make_int2(r, s);
+        for (int k = 0; k < n_pf; ++k) // heaviest (last) q-tile of the request first
+            p.pf_tiles[carry_pf + ep + k] = make_int2(r, n_pf - 1 - k);
+        if (red)
+            p.red_list[carry_red + er] = r;
+        carry_dec += td;
+        carry_pf += tp;
+        carry_red += tr;
+    }
+    if (threadIdx.x == 0) {
+        hdr->n_dec_units = (uint32_t)carry_dec;
+        hdr->n_pf_tiles = (uint32_t)carry_pf;
+        hdr->n_reduce = (uint32_t)carry_red;
+    }
+}
+
+// One warp merges the n parts of one (row, head).  o points at part 0's D
+// floats (parts o_stride floats apart), lse at part 0 (lse_stride apart).
+template <int D>
+__device__ __forceinline__ void merge_one(const float *__restrict__ o, int64_t o_stride, const float *__restrict__ lse,
+                                          int lse_stride, int n, __nv_bfloat16 *__restrict__ out, float *lse_out)
+{
+    constexpr int kPer = D / 32; // 4 (D=128) or 2 (D=64) consecutive floats per lane
+    const int lane = threadIdx.x & 31;
+    float mx = -CUDART_INF_F;
+    for (int s = lane; s < n; s += 32)
+        mx = fmaxf(mx, lse[(int64_t)s * lse_stride]);
+#pragma unroll
+    for (int o2 = 16; o2; o2 >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+        acc[i] = 0.f;
+    float z = 0.f;
+    if (mx != -CUDART_INF_F) {
+        for (int s0 = 0; s0 < n; s0 += 32) {
+            const int s = s0 + lane;
+            const float w = s < n ? __expf(lse[(int64_t)s * lse_stride] - mx) : 0.f;
+            z += w;
+            const int cnt = min(32, n - s0);
+            for (int k = 0; k < cnt; ++k) {
+                const float wk = __shfl_sync(0xffffffffu, w, k);
+                const float *src = o + (int64_t)(s0 + k) * o_stride + lane * kPer;
+                if constexpr (kPer == 4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(src);
+                    acc[0] += wk * v.x;
+                    acc[1] += wk * v.y;
+                    acc[2] += wk * v.z;
+                    acc[3] += wk * v.w;
+                } else {
+                    const float2 v = *reinterpret_cast<const float2 *>(src);
+                    acc[0] += wk * v.x;
+                    acc[1] += wk * v.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int o2 = 16; o2; o2 >>= 1)
+            z += __shfl_xor_sync(0xffffffffu, z, o2);
+    }
+    const float inv = z > 0.f ? 1.f / z : 0.f;
+    __nv_bfloat16 *dst = out + lane * kPer;
+    if constexpr (kPer == 4) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+        __nv_bfloat162 b = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+        uint2 v;
+        v.x = *reinterpret_cast<uint32_t *>(&a);
+        v.y = *reinterpret_cast<uint32_t *>(&b);
+        *reinterpret_cast<uint2 *>(dst) = v;
+    } else {
+        *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+    }
+    if (lse_out && lane == 0)
+        *lse_out = z > 0.f ? mx + logf(z) : -CUDART_INF_F;
+}
+
+// Split-KV reduce of the decode requests that were split (one CTA each).
+template <int D>
+__global__ void __launch_bounds__(256) reduce_kernel(const AttnParams p)
+{
+    const int b = blockIdx.x;
+    if (b >= (int)p.hdr->n_reduce)
+        return;
+    const int r = p.red_list[b];
+    const int qs = p.qsl[r];
+    const int q_len = p.qsl[r + 1] - qs;
+    const int L = p.seq_lens[r];
+    const int n = (L + p.split_tokens - 1) / p.split_tokens;
+    const int warps = blockDim.x >> 5;
+    for (int pair = threadIdx.x >> 5; pair < q_len * p.Hq; pair += warps) {
+        const int i = pair / p.Hq, hq = pair - i * p.Hq;
+        const int64_t idx = (((int64_t)r * p.QD + i) * p.Hq + hq) * p.max_splits;
+        const int64_t orow = (int64_t)(qs + i) * p.Hq + hq;
+        merge_one<D>(p.part_o + idx * D, D, p.part_lse + idx, 1, n, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) merge_states_kernel(const float *__restrict__ part_out,
+                                                           const float *__restrict__ part_lse,
+                                                           const int32_t *__restrict__ parts_per_row, int num_rows,
+                                                           int num_heads, int num_parts, __nv_bfloat16 *out,
+                                                           float *lse_out)
+{
+    const int64_t pair = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (pair >= (int64_t)num_rows * num_heads)
+        return;
+    const int row = (int)(pair / num_heads);
+    int n = num_parts;
+    if (parts_per_row)
+        n = max(0, min(num_parts, parts_per_row[row]));
+    merge_one<D>(part_out + pair * num_parts * D, D, part_lse + pair * num_parts, 1, n, out + pair * D,
+                 lse_out ? lse_out + pair : nullptr);
+}
+
+} // namespace
+
+cudaError_t launch_plan(const AttnParams &p, cudaStream_t s)
+{
+    plan_kernel<<<1, 1024, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reduce(const AttnParams &p, cudaStream_t s)
+{
+    if (p.D == 128)
+        reduce_kernel<128><<<p.num_seqs, 256, 0, s>>>(p);
+    else
+        reduce_kernel<64><<<p.num_seqs, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_merge_states(const float *part_out, const float *part_lse, const int32_t *parts_per_row,
+                                int num_rows, int num_heads, int num_parts, int D, void *out, float *lse_out,
+                                cudaStream_t s)
+{
+    const int64_t pairs = (int64_t)num_rows * num_heads;
+    const unsigned blocks = (unsigned)((pairs + 7) / 8);
+    auto *o = static_cast<__nv_bfloat16 *>(out);
+    if (D == 128)
+        merge_states_kernel<128><<<blocks, 256, 0, s>>>(part_out, part_lse, parts_per_row, num_rows, num_heads,
+                                                         num_parts, o, lse_out);
+    else
+        merge_states_kernel<64><<<blocks, 256, 0, s>>>(part_out, part_lse, parts_per_row, num_rows, num_heads,
+                                                        num_parts, o, lse_out);
+    return cudaGetLastError();
+}
+
+} // namespace pa

@@ -1,0 +1,112 @@
+"""Helpers shared by the GPU parity tests: move seeded workloads to the device,
+run the CUDA path through the C ABI, run the oracle on the same inputs, and
+measure the difference.  Marshalling only -- no attention arithmetic here.
+
+Parity gate (from the stated target: max-abs 2e-2, max-rel 1e-2 on bf16
+outputs computed with fp32 accumulation):
+  * max_abs  = max over all elements |gpu - oracle|                 <= 2e-2
+  * max_rel  = max over (token, head) rows of
+               max_d |gpu - oracle| / max(max_d |oracle|, 1e-2)     <= 1e-2
+    i.e. the error of each head's output vector relative to that vector's
+    magnitude (a per-element ratio is meaningless for outputs near zero);
+  * lse: max |gpu - oracle| <= 1e-3.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+from paged_kv_cache_461_b200 import api
+from paged_kv_cache_461_b200 import workloads as W
+
+ATOL = 2e-2
+RTOL = 1e-2
+LSE_TOL = 1e-3
+
+
+def to_dev_bf16(a: np.ndarray, dev="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def to_host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+class DevStep:
+    """Device copies of one step (metadata + values)."""
+
+    def __init__(self, layout: W.StepLayout, vals: W.StepValues, dev="cuda"):
+        self.layout = layout
+        self.qsl = torch.from_numpy(layout.query_start_loc).to(dev)
+        self.seq_lens = torch.from_numpy(layout.seq_lens).to(dev)
+        self.bt = torch.from_numpy(layout.block_table).to(dev)
+        self.slots = torch.from_numpy(layout.slot_mapping).to(dev)
+        if isinstance(vals.q, np.ndarray):
+            self.q, self.k_new, self.v_new = (to_dev_bf16(x, dev) for x in (vals.q, vals.k_new, vals.v_new))
+            self.k_cache, self.v_cache = to_dev_bf16(vals.k_cache, dev), to_dev_bf16(vals.v_cache, dev)
+        else:
+            self.q, self.k_new, self.v_new = vals.q, vals.k_new, vals.v_new
+            self.k_cache, self.v_cache = vals.k_cache, vals.v_cache
+
+    def write(self):
+        api.kv_write(self.k_new, self.v_new, self.slots, self.k_cache, self.v_cache)
+
+    def attend(self, kv_split_tokens=0, with_lse=True, scale=None, workspace=None):
+        lay = self.layout
+        lse = torch.full((lay.num_tokens, lay.num_q_heads), float("nan"), dtype=torch.float32,
+                         device=self.q.device) if with_lse else None
+        out = torch.full_like(self.q, float("nan"))
+        if workspace is None:
+            workspace = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, self.k_cache,
+                                            lay.max_seq_len, kv_split_tokens)
+        api.attention_mixed(self.q, self.k_cache, self.v_cache, self.qsl, self.seq_lens, self.bt,
+                            lay.max_query_len, lay.max_seq_len, softmax_scale=scale, out=out, lse=lse,
+                            workspace=workspace, kv_split_tokens=kv_split_tokens)
+        self.workspace = workspace
+        return out, lse
+
+
+def oracle_for_step(layout: W.StepLayout, vals: W.StepValues, scale=None, token_list=None):
+    """Oracle on the host copy of the inputs (KV written by the oracle's own write)."""
+    kc, vc = oracle.kv_write(vals.k_new, vals.v_new, layout.slot_mapping, vals.k_cache, vals.v_cache)
+    if scale is None:
+        scale = 1.0 / math.sqrt(layout.head_dim)
+    return oracle.attention_for(layout, kc, vc, vals.q, scale=scale, token_list=token_list)
+
+
+def errors(gpu_out: torch.Tensor, ref: np.ndarray, rows=None) -> dict:
+    g = bf16_to_f64(gpu_out)
+    if rows is not None:
+        g = g[rows]
+    d = np.abs(g - ref)
+    if d.size == 0:
+        return {"max_abs": 0.0, "max_rel": 0.0, "nan": False}
+    nan = bool(np.isnan(g).any())
+    row_err = d.max(axis=-1)
+    row_mag = np.maximum(np.abs(ref).max(axis=-1), 1e-2)
+    rel = row_err / row_mag
+    i = np.unravel_index(int(np.nanargmax(d)), d.shape)
+    return {"max_abs": float(np.nanmax(d)), "max_rel": float(np.nanmax(rel)), "argmax": tuple(int(x) for x in i),
+            "nan": nan}
+
+
+def assert_parity(gpu_out, ref, gpu_lse=None, ref_lse=None, rows=None, what=""):
+    e = errors(gpu_out, ref, rows)
+    assert not e["nan"], f"{what}: NaN in GPU output"
+    assert e["max_abs"] <= ATOL, f"{what}: max_abs {e}"
+    assert e["max_rel"] <= RTOL, f"{what}: max_rel {e}"
+    if gpu_lse is not None and ref_lse is not None:
+        gl = gpu_lse.cpu().numpy().astype(np.float64)
+        if rows is not None:
+            gl = gl[rows]
+        dl = np.abs(gl - ref_lse)
+        assert not np.isnan(gl).any(), f"{what}: NaN in GPU lse"
+        assert dl.max() <= LSE_TOL, f"{what}: lse err {dl.max()}"
+    return e

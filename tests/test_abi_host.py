@@ -1,0 +1,141 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every entry
+point include/pa.h declares, and rejects bad arguments on the host before any
+CUDA call (no compute is launched in these tests)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from paged_kv_cache_461_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return api.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert sorted(api.EXPORTED) == declared_symbols()
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", api.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\s(pa_[a-z_0-9]+)$", out, flags=re.M))
+    for sym in declared_symbols():
+        assert sym in exported, f"{sym} declared in pa.h but not exported"
+        assert getattr(L, sym) is not None
+
+
+def test_library_exports_nothing_else(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", api.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    ours = set(re.findall(r"\s(pa_[a-z_0-9]+)$", out, flags=re.M))
+    assert ours == set(declared_symbols())
+
+
+def test_version_and_status_strings(L):
+    assert L.pa_abi_version() == 1
+    for code, name in api.STATUS_NAMES.items():
+        assert L.pa_status_string(code).decode() == name
+
+
+def _desc(nb=64, hkv=8, d=128, bs=16):
+    return api.CacheDesc(nb, hkv, d, bs)
+
+
+def test_workspace_size_rules(L):
+    d = _desc()
+    ws = lambda *a: L.pa_workspace_size(*a)
+    base = ws(4, 4, 32, ctypes.byref(d), 1000)
+    assert base > 0
+    # grows (never shrinks) with every bound
+    assert ws(8, 4, 32, ctypes.byref(d), 1000) >= base
+    assert ws(4, 400, 32, ctypes.byref(d), 1000) >= base
+    assert ws(4, 4, 32, ctypes.byref(d), 100000) >= base
+    # invalid / unsupported -> 0
+    assert ws(4, 4, 30, ctypes.byref(d), 1000) == 0          # Hq % Hkv != 0
+    assert ws(-1, 4, 32, ctypes.byref(d), 1000) == 0
+    assert ws(4, 4, 32, ctypes.byref(_desc(d=96)), 1000) == 0
+    assert ws(4, 4, 32, ctypes.byref(_desc(bs=32)), 1000) == 0
+    assert ws(4, 4, 3 * 8, ctypes.byref(d), 1000) == 0       # G = 3 does not divide 128
+    # a split size must be a multiple of 16
+    o = api.AttnOptions()
+    o.kv_split_tokens = 24
+    assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) == 0
+    o.kv_split_tokens = 32
+    assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) > base
+    o.reserved[0] = 1
+    assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) == 0
+
+
+FAKE = 1 << 40  # a non-null pointer value; never dereferenced by host validation paths below
+
+
+def test_kv_write_host_validation(L):
+    d = _desc()
+    call = lambda *a: L.pa_kv_write(*a)
+    assert call(FAKE, FAKE, 1024, FAKE, 0, FAKE, FAKE, ctypes.byref(d), None) == 0          # nothing to do
+    assert call(None, FAKE, 1024, FAKE, 4, FAKE, FAKE, ctypes.byref(d), None) == 1          # null k_new
+    assert call(FAKE, FAKE, 1024, None, 4, FAKE, FAKE, ctypes.byref(d), None) == 1          # null slots
+    assert call(FAKE, FAKE, 1000, FAKE, 4, FAKE, FAKE, ctypes.byref(d), None) == 1          # row stride < Hkv*D
+    assert call(FAKE, FAKE, 1024, FAKE, -1, FAKE, FAKE, ctypes.byref(d), None) == 1
+    assert call(FAKE, FAKE, 1024, FAKE, 4, FAKE, FAKE, None, None) == 1                     # no descriptor
+    assert call(FAKE, FAKE, 1024, FAKE, 4, FAKE, FAKE, ctypes.byref(_desc(d=80)), None) == 2
+    assert call(FAKE, FAKE, 1024, FAKE, 4, FAKE, FAKE, ctypes.byref(_desc(bs=8)), None) == 2
+    assert call(FAKE, FAKE, 1024, FAKE, 4, FAKE, FAKE, ctypes.byref(_desc(nb=1 << 30)), None) == 2
+
+
+def _attn(L, **kw):
+    a = dict(q=FAKE, hq=32, k=FAKE, v=FAKE, desc=_desc(), qsl=FAKE, sl=FAKE, bt=FAKE, bts=64, R=4, T=4, mq=1,
+             ms=1000, scale=0.088, out=FAKE + (1 << 30), lse=None, ws=FAKE + (1 << 32), wsb=1 << 30)
+    a.update(kw)
+    return L.pa_attention_mixed(a["q"], a["hq"], a["k"], a["v"], ctypes.byref(a["desc"]), a["qsl"], a["sl"], a["bt"],
+                                a["bts"], a["R"], a["T"], a["mq"], a["ms"], ctypes.c_float(a["scale"]), a["out"],
+                                a["lse"], a["ws"], a["wsb"], None)
+
+
+def test_attention_host_validation(L):
+    assert _attn(L, R=0) == 0 and _attn(L, T=0) == 0       # empty step: nothing enqueued
+    assert _attn(L, q=None) == 1
+    assert _attn(L, bt=None) == 1
+    assert _attn(L, hq=30) == 1                            # Hq % Hkv
+    assert _attn(L, bts=10) == 1                           # bt_stride < ceil(max_seq_len / 16)
+    assert _attn(L, R=-1) == 1
+    assert _attn(L, mq=-1) == 1
+    assert _attn(L, scale=float("nan")) == 1
+    assert _attn(L, out=FAKE) == 1                         # out aliases q
+    assert _attn(L, out=FAKE + 100) == 1                   # partial overlap
+    assert _attn(L, desc=_desc(d=256)) == 2
+    assert _attn(L, hq=8 * 3) == 2                         # G = 3
+    assert _attn(L, q=FAKE + 2) == 2                       # q not 16-byte aligned
+    assert _attn(L, wsb=16) == 3                           # workspace too small
+
+
+def test_merge_and_gather_host_validation(L):
+    assert L.pa_merge_attn_states(FAKE, FAKE, None, 4, 8, 3, 96, FAKE, None, None) == 2
+    assert L.pa_merge_attn_states(FAKE, FAKE, None, -1, 8, 3, 128, FAKE, None, None) == 1
+    assert L.pa_merge_attn_states(FAKE, FAKE, None, 0, 8, 3, 128, FAKE, None, None) == 0
+    assert L.pa_merge_attn_states(None, FAKE, None, 4, 8, 3, 128, FAKE, None, None) == 1
+    assert L.pa_debug_gather_kv(FAKE, ctypes.byref(_desc()), FAKE, -3, FAKE, None) == 1
+    assert L.pa_debug_gather_kv(FAKE, ctypes.byref(_desc()), FAKE, 0, FAKE, None) == 0
+    assert L.pa_build_slot_mapping(None, FAKE, FAKE, 4, 2, 8, FAKE, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        api.lib()

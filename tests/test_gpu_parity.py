@@ -1,0 +1,418 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, on the same seeded inputs.
+
+Bit-exact: KV write, slot mapping, gather.  Within the parity gate of
+gpu_util (max-abs 2e-2, per-head-vector relative 1e-2, lse 1e-3): decode,
+split-KV, merge, prefill, mixed steps, stress inputs and the five full-size
+workloads on sampled rows.  Invariances the pages state are checked on the
+GPU too: block-id permutation and shared-vs-private prefix blocks must give
+bit-identical outputs, chunked prefill and split/unsplit must agree within
+the gate.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_461_b200 import api, build
+from paged_kv_cache_461_b200 import workloads as W
+from tests.gpu_util import DevStep, assert_parity, bf16_to_f64, errors, oracle_for_step, to_dev_bf16, to_host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    build.build()
+    api.lib()
+    torch.manual_seed(0)
+
+
+def _layout(name, ctx, q, Hq, Hkv, D, seed, extra_blocks=17, shared=0):
+    ctx = np.asarray(ctx)
+    q = np.asarray(q)
+    need = sum((int(c) + int(k) + 15) // 16 for c, k in zip(ctx, q))
+    return W.build_layout(name, ctx, q, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, num_blocks=need + extra_blocks,
+                          seed=seed, shared_prefix_tokens=shared)
+
+
+def _run(lay, vals=None, split=0, scale=None, **vk):
+    if vals is None:
+        vals = W.make_values_numpy(lay, **vk)
+    st = DevStep(lay, vals)
+    st.write()
+    out, lse = st.attend(kv_split_tokens=split, scale=scale)
+    torch.cuda.synchronize()
+    ref, ref_lse, _ = oracle_for_step(lay, vals, scale=scale)
+    return st, out, lse, ref, ref_lse
+
+
+# ----------------------------------------------------------------------------- bit-exact data movement
+
+@pytest.mark.parametrize("D,Hkv,T", [(64, 4, 7), (128, 8, 256), (128, 1, 33), (64, 2, 1000)])
+def test_kv_write_bit_exact(D, Hkv, T):
+    rng = np.random.default_rng(D + Hkv + T)
+    ctx = rng.integers(0, 60, size=T)
+    lay = _layout("w", ctx, np.ones(T, np.int32), Hkv, Hkv, D, seed=T)
+    vals = W.make_values_numpy(lay, sentinel="pattern")
+    slots = lay.slot_mapping.copy()
+    slots[rng.random(T) < 0.2] = -1                       # padding tokens
+    st = DevStep(lay, vals)
+    st.slots = torch.from_numpy(slots).cuda()
+    st.write()
+    kc, vc = oracle.kv_write(vals.k_new, vals.v_new, slots, vals.k_cache, vals.v_cache)
+    assert np.array_equal(to_host_bits(st.k_cache), kc)
+    assert np.array_equal(to_host_bits(st.v_cache), vc)
+
+
+def test_kv_write_from_fused_qkv_rows():
+    T, Hq, Hkv, D = 50, 32, 8, 128
+    lay = _layout("fused", np.arange(T) % 40, np.ones(T, np.int32), Hq, Hkv, D, seed=5)
+    vals = W.make_values_numpy(lay, sentinel="pattern")
+    qkv = np.zeros((T, (Hq + 2 * Hkv) * D), np.uint16)
+    qkv[:, Hq * D:(Hq + Hkv) * D] = vals.k_new.reshape(T, -1)
+    qkv[:, (Hq + Hkv) * D:] = vals.v_new.reshape(T, -1)
+    qkv_d = to_dev_bf16(qkv)
+    k_view = qkv_d[:, Hq * D:(Hq + Hkv) * D].view(T, Hkv, D)
+    v_view = qkv_d[:, (Hq + Hkv) * D:].view(T, Hkv, D)
+    st = DevStep(lay, vals)
+    api.kv_write(k_view, v_view, st.slots, st.k_cache, st.v_cache)
+    kc, vc = oracle.kv_write(vals.k_new, vals.v_new, lay.slot_mapping, vals.k_cache, vals.v_cache)
+    assert np.array_equal(to_host_bits(st.k_cache), kc) and np.array_equal(to_host_bits(st.v_cache), vc)
+
+
+def test_kv_write_unaligned_rows_take_the_scalar_path():
+    T, Hkv, D = 9, 2, 64
+    lay = _layout("odd", np.arange(T), np.ones(T, np.int32), Hkv, Hkv, D, seed=6)
+    vals = W.make_values_numpy(lay, sentinel="pattern")
+    buf = np.zeros((T, Hkv * D + 1), np.uint16)          # odd row stride: no 16-byte vectors
+    buf[:, 1:] = vals.k_new.reshape(T, -1)
+    bufv = np.zeros_like(buf)
+    bufv[:, 1:] = vals.v_new.reshape(T, -1)
+    kd, vd = to_dev_bf16(buf), to_dev_bf16(bufv)
+    st = DevStep(lay, vals)
+    d = api.cache_desc(st.k_cache)
+    import ctypes
+    rc = api.lib().pa_kv_write(kd.data_ptr() + 2, vd.data_ptr() + 2, Hkv * D + 1, st.slots.data_ptr(), T,
+                               st.k_cache.data_ptr(), st.v_cache.data_ptr(), ctypes.byref(d), None)
+    assert rc == 0
+    torch.cuda.synchronize()
+    kc, vc = oracle.kv_write(vals.k_new, vals.v_new, lay.slot_mapping, vals.k_cache, vals.v_cache)
+    assert np.array_equal(to_host_bits(st.k_cache), kc) and np.array_equal(to_host_bits(st.v_cache), vc)
+
+
+def test_slot_mapping_bit_exact():
+    rng = np.random.default_rng(2)
+    ctx = rng.integers(0, 500, size=40)
+    q = rng.integers(0, 70, size=40)
+    lay = _layout("slots", ctx, q, 8, 8, 64, seed=3)
+    st = DevStep(lay, W.make_values_numpy(lay))
+    got = api.build_slot_mapping(st.qsl, st.seq_lens, st.bt, lay.num_tokens).cpu().numpy()
+    assert np.array_equal(got, oracle.slot_mapping(lay.query_start_loc, lay.seq_lens, lay.block_table))
+
+
+def test_debug_gather_bit_exact():
+    lay = _layout("g", [0, 15, 16, 17, 300], [1, 1, 1, 1, 1], 8, 2, 128, seed=4)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    kc, _ = oracle.kv_write(vals.k_new, vals.v_new, lay.slot_mapping, vals.k_cache, vals.v_cache)
+    for r in range(lay.num_seqs):
+        L = int(lay.seq_lens[r])
+        got = to_host_bits(api.debug_gather_kv(st.k_cache, st.bt[r], L))
+        assert np.array_equal(got, oracle.gather_kv(kc, lay.block_table[r], L))
+
+
+# ----------------------------------------------------------------------------- decode
+
+def test_tiny_decode_workload():
+    lay = W.workload_layout("tiny_decode")
+    st, out, lse, ref, ref_lse = _run(lay)
+    assert_parity(out, ref, lse, ref_lse, what="tiny_decode")
+
+
+DECODE_CASES = [
+    # (D, Hq, Hkv, q_len, split)
+    (128, 32, 8, 1, 0), (128, 32, 8, 1, 64), (128, 32, 8, 2, 0), (128, 32, 8, 2, 32),
+    (128, 64, 8, 1, 0), (128, 64, 8, 1, 256), (128, 8, 8, 1, 0), (128, 8, 8, 8, 48),
+    (64, 4, 4, 1, 0), (64, 16, 4, 2, 16), (64, 8, 1, 1, 0), (128, 32, 2, 1, 0), (128, 32, 2, 1, 80),
+    (128, 16, 8, 4, 0), (64, 128, 8, 1, 0),
+]
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,q_len,split", DECODE_CASES)
+def test_decode_parity(D, Hq, Hkv, q_len, split):
+    rng = np.random.default_rng(D * 7 + Hq + q_len + split)
+    ctx = np.concatenate([rng.integers(0, 700, size=9), [0, 15, 16, 17, 31, 1023 if split else 64]])
+    ctx = np.maximum(ctx, 0)
+    lay = _layout("dec", ctx, np.full(len(ctx), q_len, np.int32), Hq, Hkv, D, seed=int(ctx.sum()) % 1000)
+    st, out, lse, ref, ref_lse = _run(lay, split=split)
+    assert_parity(out, ref, lse, ref_lse, what=f"decode D{D} Hq{Hq} Hkv{Hkv} q{q_len} split{split}")
+    assert api.read_device_status(st.workspace) == 0
+
+
+def test_merge_attn_states_matches_oracle_merge():
+    rng = np.random.default_rng(8)
+    N, H, S, D = 6, 4, 9, 128
+    o = rng.standard_normal((N, H, S, D)).astype(np.float32)
+    lse = (rng.standard_normal((N, H, S)) * 4).astype(np.float32)
+    lse[0, 0, 3] = -np.inf                              # an empty part
+    lse[1, 1, :] = -np.inf                              # a row with no keys at all
+    parts = np.array([9, 9, 1, 5, 9, 0], np.int32)
+    out_d = api.merge_attn_states(torch.from_numpy(o).cuda(), torch.from_numpy(lse).cuda(),
+                                  torch.from_numpy(parts).cuda(),
+                                  lse_out=(lse_d := torch.empty((N, H), device="cuda")))
+    got = bf16_to_f64(out_d)
+    for i in range(N):
+        for h in range(H):
+            n = parts[i]
+            ref, rl = oracle.merge_states(o[i, h, :n].astype(np.float64), lse[i, h, :n].astype(np.float64))
+            assert np.abs(got[i, h] - ref).max() <= 1e-2 * max(np.abs(ref).max(), 1e-2)
+            gl = float(lse_d[i, h])
+            assert (gl == rl == -math.inf) or abs(gl - rl) < 1e-3
+
+
+# ----------------------------------------------------------------------------- prefill / mixed
+
+PREFILL_CASES = [
+    # (D, Hq, Hkv, ctx list, q list)
+    (128, 32, 8, [0, 0, 33, 200], [5, 130, 47, 300]),
+    (128, 32, 8, [1000, 17], [129, 256]),
+    (128, 8, 8, [0, 5, 130], [128, 1, 257]),
+    (64, 8, 8, [0, 140], [200, 77]),
+    (64, 32, 4, [31, 0], [64, 3]),
+    (128, 64, 8, [0, 250], [17, 40]),
+    (128, 16, 16, [48, 0, 0], [100, 16, 2]),
+    (128, 128, 1, [7, 0], [3, 2]),
+]
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,ctx,q", PREFILL_CASES)
+def test_prefill_parity(D, Hq, Hkv, ctx, q):
+    lay = _layout("pf", ctx, q, Hq, Hkv, D, seed=sum(ctx) + sum(q))
+    st, out, lse, ref, ref_lse = _run(lay)
+    assert_parity(out, ref, lse, ref_lse, what=f"prefill D{D} Hq{Hq} Hkv{Hkv} ctx{ctx} q{q}")
+    assert api.read_device_status(st.workspace) == 0
+
+
+def _mixed_layout(seed, n_dec=24, chunks=((300, 0), (129, 700), (64, 1500), (1, 40)), D=128, Hq=32, Hkv=8,
+                  shuffle=False):
+    rng = np.random.default_rng(seed)
+    dec_ctx = rng.integers(0, 2000, size=n_dec)
+    ctx = list(dec_ctx) + [c for _, c in chunks]
+    q = [1] * n_dec + [n for n, _ in chunks]
+    if shuffle:
+        order = rng.permutation(len(ctx))
+        ctx = [ctx[i] for i in order]
+        q = [q[i] for i in order]
+    return _layout("mixed", ctx, q, Hq, Hkv, D, seed=seed)
+
+
+@pytest.mark.parametrize("shuffle", [False, True])
+def test_mixed_step_parity(shuffle):
+    lay = _mixed_layout(11, shuffle=shuffle)
+    st, out, lse, ref, ref_lse = _run(lay)
+    assert_parity(out, ref, lse, ref_lse, what=f"mixed shuffle={shuffle}")
+
+
+@pytest.mark.parametrize("kind", ["q_x8", "v_mean3", "ctx_1_mod_16"])
+def test_stress_inputs(kind):
+    if kind == "ctx_1_mod_16":
+        # every sequence ends one token into a fresh block (partial last blocks everywhere)
+        rng = np.random.default_rng(12)
+        q = np.array([1] * 16 + [40, 130, 7], np.int32)
+        L = rng.integers(1, 120, size=len(q)) * 16 + 1
+        lay = _layout("c1", L - q, q, 32, 8, 128, seed=12)
+        vk = {}
+    else:
+        lay = _mixed_layout(13)
+        vk = {"q_scale": 8.0} if kind == "q_x8" else {"v_mean": 3.0}
+    st, out, lse, ref, ref_lse = _run(lay, **vk)
+    assert_parity(out, ref, lse, ref_lse, what=kind)
+
+
+def test_empty_requests_and_padding_rows_are_left_alone():
+    lay = _layout("e", [10, 40, 0, 300], [0, 1, 0, 70], 32, 8, 128, seed=14)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    out, lse = st.attend()
+    torch.cuda.synchronize()
+    ref, ref_lse, _ = oracle_for_step(lay, vals)
+    assert_parity(out, ref, lse, ref_lse, what="empty requests")
+
+
+# ----------------------------------------------------------------------------- invariances on the GPU
+
+def test_block_permutation_gives_bit_identical_output():
+    lay = _mixed_layout(21)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    out1, lse1 = st.attend()
+    perm = np.random.default_rng(3).permutation(lay.num_blocks)
+    lay2 = W.permute_physical_blocks(lay, perm)
+    vals2 = W.permute_pool_numpy(vals, perm)
+    st2 = DevStep(lay2, vals2)
+    st2.write()
+    out2, lse2 = st2.attend()
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(lse1, lse2)
+
+
+def test_shared_prefix_blocks_equal_private_copies_bit_exactly():
+    rng = np.random.default_rng(22)
+    suffix = rng.integers(64, 300, size=12)
+    lay = W.build_layout("share", 512 + suffix, np.ones(12, np.int32), num_q_heads=32, num_kv_heads=8,
+                         head_dim=128, num_blocks=1200, rng=rng, seed=22, shared_prefix_tokens=512)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    out1, lse1 = st.attend()
+    lay2, copies = W.privatize_shared_prefix(lay)
+    vals2 = W.copy_blocks_numpy(vals, copies)
+    st2 = DevStep(lay2, vals2)
+    st2.write()
+    out2, lse2 = st2.attend()
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    ref, ref_lse, _ = oracle_for_step(lay, vals)
+    assert_parity(out1, ref, lse1, ref_lse, what="shared prefix")
+
+
+def test_mixed_step_equals_requests_run_alone_bit_exactly():
+    lay = _mixed_layout(23, n_dec=6)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    out, _ = st.attend()
+    qsl = lay.query_start_loc
+    for r in range(lay.num_seqs):
+        sub = W.StepLayout("one", lay.num_q_heads, lay.num_kv_heads, lay.head_dim, lay.num_blocks,
+                           lay.q_lens[r:r + 1], lay.ctx_lens[r:r + 1], lay.block_table[r:r + 1])
+        s1 = DevStep(sub, W.StepValues(vals.q[qsl[r]:qsl[r + 1]], vals.k_new[qsl[r]:qsl[r + 1]],
+                                       vals.v_new[qsl[r]:qsl[r + 1]], vals.k_cache, vals.v_cache))
+        s1.write()
+        o1, _ = s1.attend()
+        assert torch.equal(o1.view(torch.int16), out[qsl[r]:qsl[r + 1]].view(torch.int16)), f"request {r}"
+
+
+def test_chunked_prefill_matches_one_shot_within_gate():
+    n, Hq, Hkv, D = 700, 32, 8, 128
+    one = _layout("one", [0], [n], Hq, Hkv, D, seed=24)
+    vals = W.make_values_numpy(one)
+    st = DevStep(one, vals)
+    st.write()
+    full, _ = st.attend()
+    kc = to_dev_bf16(vals.k_cache)
+    vc = to_dev_bf16(vals.v_cache)
+    pos = 0
+    rows = []
+    for chunk in (129, 300, 1, 270):
+        lay = W.StepLayout("chunk", Hq, Hkv, D, one.num_blocks, np.array([chunk], np.int32),
+                           np.array([pos], np.int32), one.block_table)
+        sl = slice(pos, pos + chunk)
+        s = DevStep(lay, W.StepValues(vals.q[sl], vals.k_new[sl], vals.v_new[sl], vals.k_cache, vals.v_cache))
+        s.k_cache, s.v_cache = kc, vc            # one cache, written chunk by chunk
+        s.write()
+        o, _ = s.attend()
+        rows.append(o)
+        pos += chunk
+    chunked = torch.cat(rows)
+    ref, _, _ = oracle_for_step(one, vals)
+    assert_parity(chunked, ref, what="chunked")
+    e = errors(chunked, bf16_to_f64(full))
+    assert e["max_abs"] <= 2e-2 and e["max_rel"] <= 1e-2
+
+
+def test_split_and_unsplit_decode_agree():
+    rng = np.random.default_rng(25)
+    ctx = rng.integers(1000, 5000, size=20)
+    lay = _layout("split", ctx, np.ones(20, np.int32), 64, 8, 128, seed=25)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    a, la = st.attend(kv_split_tokens=16 * 400)   # one split for every request
+    b, lb = st.attend(kv_split_tokens=128)        # up to 40 splits
+    e = errors(a, bf16_to_f64(b))
+    assert e["max_abs"] <= 2e-2 and e["max_rel"] <= 1e-2
+    assert (la - lb).abs().max().item() <= 1e-3
+
+
+# ----------------------------------------------------------------------------- device-side checks
+
+def test_bad_metadata_sets_status_and_never_faults():
+    lay = _mixed_layout(26, n_dec=4)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    good, _ = st.attend()
+    # seq_len beyond max_seq_len for request 1 -> skipped, flagged
+    bad_lens = st.seq_lens.clone()
+    bad_lens[1] = lay.max_seq_len + 5
+    out = torch.zeros_like(st.q)
+    ws = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, st.k_cache, lay.max_seq_len)
+    api.attention_mixed(st.q, st.k_cache, st.v_cache, st.qsl, bad_lens, st.bt, lay.max_query_len, lay.max_seq_len,
+                        out=out, workspace=ws)
+    assert api.read_device_status(ws) & api.DEVICE_BAD_SEQ
+    qsl = lay.query_start_loc
+    assert torch.equal(out[qsl[1]:qsl[2]], torch.zeros_like(out[qsl[1]:qsl[2]]))
+    assert torch.equal(out[qsl[2]:].view(torch.int16), good[qsl[2]:].view(torch.int16))
+    # a block id outside the pool reads zeros and is flagged
+    bt = st.bt.clone()
+    bt[0, 0] = lay.num_blocks + 1000
+    api.attention_mixed(st.q, st.k_cache, st.v_cache, st.qsl, st.seq_lens, bt, lay.max_query_len, lay.max_seq_len,
+                        out=out, workspace=ws)
+    assert api.read_device_status(ws) & api.DEVICE_BAD_BLOCK
+    # and the next good call clears the word
+    api.attention_mixed(st.q, st.k_cache, st.v_cache, st.qsl, st.seq_lens, st.bt, lay.max_query_len,
+                        lay.max_seq_len, out=out, workspace=ws)
+    assert api.read_device_status(ws) == 0
+
+
+# ----------------------------------------------------------------------------- the five workloads, full size
+
+def _sub_problem(lay: W.StepLayout, req_ids, k_host_pool, v_host_pool, q_host, k_new_host, v_new_host):
+    """Restrict a step to some requests with a compact copy of their blocks (relabelled)."""
+    req_ids = np.asarray(sorted(req_ids))
+    nblk = (lay.seq_lens[req_ids] + 15) // 16
+    ids = np.unique(np.concatenate([lay.block_table[r, :n] for r, n in zip(req_ids, nblk)]))
+    remap = np.full(lay.num_blocks, -1, np.int64)
+    remap[ids] = np.arange(len(ids))
+    bt = np.full((len(req_ids), lay.bt_stride), -1, np.int32)
+    for i, (r, n) in enumerate(zip(req_ids, nblk)):
+        bt[i, :n] = remap[lay.block_table[r, :n]]
+    sub = W.StepLayout(lay.name + "_sub", lay.num_q_heads, lay.num_kv_heads, lay.head_dim, len(ids),
+                       lay.q_lens[req_ids], lay.ctx_lens[req_ids], bt)
+    qsl = lay.query_start_loc
+    rows = np.concatenate([np.arange(qsl[r], qsl[r + 1]) for r in req_ids]).astype(np.int64)
+    vals = W.StepValues(q_host[rows], k_new_host[rows], v_new_host[rows], k_host_pool(ids), v_host_pool(ids))
+    return sub, vals, rows
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "mixed_step_8192", "prefix_sharing", "long_context_decode"])
+def test_full_size_workload_on_sampled_rows(name):
+    lay = W.workload_layout(name)
+    vals = W.make_values_torch(lay, "cuda")
+    rng = np.random.default_rng(99)
+    R = lay.num_seqs
+    pick = set(rng.choice(R, size=min(R, 12), replace=False).tolist())
+    pick |= {0, R - 1, int(np.argmax(lay.seq_lens)), int(np.argmax(lay.q_lens))}
+    # host copies of the inputs, taken before the CUDA path writes anything
+    kpool = lambda ids: to_host_bits(vals.k_cache[torch.from_numpy(ids).cuda()])
+    vpool = lambda ids: to_host_bits(vals.v_cache[torch.from_numpy(ids).cuda()])
+    sub, svals, rows = _sub_problem(lay, pick, kpool, vpool, to_host_bits(vals.q), to_host_bits(vals.k_new),
+                                    to_host_bits(vals.v_new))
+    st = DevStep(lay, vals)
+    st.write()
+    out, lse = st.attend()
+    torch.cuda.synchronize()
+    assert api.read_device_status(st.workspace) == 0
+    # rows to check: every row of short requests, first/last/random rows of long prefill chunks
+    n = sub.num_tokens
+    tl = np.arange(n) if n <= 64 else np.unique(np.concatenate([np.arange(8), np.arange(n - 8, n),
+                                                                rng.choice(n, 48, replace=False)]))
+    ref, ref_lse, _ = oracle_for_step(sub, svals, token_list=tl)
+    assert_parity(out, ref, lse, ref_lse, rows=rows[tl], what=name)
+    assert not torch.isnan(out.float()).any()
