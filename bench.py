@@ -74,19 +74,23 @@ def _traffic(name, files):
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """nvidia-smi sampled every period_ms in the background; stop() keeps the samples that
+    arrived inside the timed window (host monotonic clock)."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int, period_ms: int = 20):
+    def __init__(self, device_index: int, period_ms: int = 10):
         self.rows = []
         self.proc = None
+        self.first = threading.Event()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", str(period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            self.first.wait(timeout=5.0)
         except OSError:
             self.proc = None
 
@@ -94,23 +98,33 @@ class ClockSampler:
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) == 7:
-                self.rows.append(parts)
+                self.rows.append((time.monotonic(), parts))
+                self.first.set()
 
-    def stop(self):
+    def stop(self, t0: float, t1: float):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.05)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.t.join(timeout=2)
-        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        inside = [r for ts, r in self.rows if t0 <= ts <= t1 + 0.02]
+        note = "samples inside the timed region"
+        if not inside:  # region shorter than the sampling period: take the samples bracketing it
+            after = [r for ts, r in self.rows if ts >= t0][:2]
+            before = [r for ts, r in self.rows if ts < t0][-1:]
+            inside = before + after
+            note = "timed region shorter than the sampling period; nearest samples"
+        num = lambda v: v.replace(".", "", 1).isdigit()
+        sm = [float(r[0]) for r in inside if num(r[0])]
+        mx = [float(r[1]) for r in inside if num(r[1])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[3 + i].lower() == "active"})
+        reasons = sorted({names[i] for r in inside for i in range(4) if r[3 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+                "reasons": reasons, "samples": len(inside), "note": note}
 
 
 # --------------------------------------------------------------------------- distributed plumbing
@@ -197,8 +211,9 @@ class Step:
         self.attention()
 
 
-def _time_region(fn, steps, warmup, ws, sub_events=None):
-    """W untimed steps, then EXACTLY `steps` steps between barrier+sync on both sides."""
+def _time_region(fn, steps, warmup, ws, window=None):
+    """W untimed steps, then EXACTLY `steps` steps between barrier+sync on both sides.
+    `window` (a list) receives the host monotonic times bracketing the timed region."""
     import torch
     for _ in range(warmup):
         fn()
@@ -207,12 +222,16 @@ def _time_region(fn, steps, warmup, ws, sub_events=None):
     stream = torch.cuda.current_stream()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    h0 = time.monotonic()
     t0.record(stream)
     for _ in range(steps):
         fn()
     t1.record(stream)
     torch.cuda.synchronize()
+    h1 = time.monotonic()
     _barrier(ws)
+    if window is not None:
+        window[:] = [h0, h1]
     return t0.elapsed_time(t1)
 
 
@@ -363,6 +382,43 @@ def reference_arm(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------- small cases for ncu captures
+
+def profile_case(kind: str, launches: int):
+    """A reduced copy of a workload for ncu (same shapes, fewer requests, pool sized to fit):
+    decode: the first 64 requests of the Llama-3-8B-shaped decode batch (~0.6 GB of KV, above L2);
+    prefill: the prefill chunks of the mixed 8192-token step alone.
+    Runs 1 warm-up launch of pa_attention_mixed and then `launches` more."""
+    import torch
+
+    from paged_kv_cache_461_b200 import api, build
+    from paged_kv_cache_461_b200 import workloads as W
+    build.build()
+    full = W.workload_layout(HEADLINE if kind == "decode" else MIXED)
+    if kind == "decode":
+        idx = np.arange(64)
+    else:
+        G = full.num_q_heads // full.num_kv_heads
+        idx = np.nonzero(full.q_lens * G > 8)[0]
+    lay = W.build_layout(f"{full.name}_{kind}_case", full.ctx_lens[idx], full.q_lens[idx],
+                         num_q_heads=full.num_q_heads, num_kv_heads=full.num_kv_heads, head_dim=full.head_dim,
+                         seed=full.seed)
+    v = W.make_values_torch(lay, "cuda")
+    qsl = torch.from_numpy(lay.query_start_loc).cuda()
+    sl = torch.from_numpy(lay.seq_lens).cuda()
+    bt = torch.from_numpy(lay.block_table).cuda()
+    slots = torch.from_numpy(lay.slot_mapping).cuda()
+    api.kv_write(v.k_new, v.v_new, slots, v.k_cache, v.v_cache)
+    ws = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, v.k_cache, lay.max_seq_len)
+    out = torch.empty_like(v.q)
+    for _ in range(1 + launches):
+        api.attention_mixed(v.q, v.k_cache, v.v_cache, qsl, sl, bt, lay.max_query_len, lay.max_seq_len,
+                            out=out, workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": kind, **lay.describe(), "kv_bytes": lay.kv_bytes(),
+                      "pool_bytes": 2 * v.k_cache.numel() * 2}))
+
+
 # --------------------------------------------------------------------------- main
 
 def main():
@@ -374,7 +430,12 @@ def main():
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="headline only (no mixed step, e2e, prefill)")
+    ap.add_argument("--profile-case", choices=["decode", "prefill"],
+                    help="run a small case of one kernel for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case, args.steps)
+        return
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     if args.impl == "reference":
@@ -394,8 +455,9 @@ def main():
 
     st = Step(args.workload)
     sampler = ClockSampler(local)
-    ms_total = _time_region(st.step, args.steps, args.warmup, ws)
-    clocks = sampler.stop()
+    win = []
+    ms_total = _time_region(st.step, args.steps, args.warmup, ws, window=win)
+    clocks = sampler.stop(*win)
     ms_total = _max_over_ranks(ms_total, ws)
     ms_step = ms_total / args.steps
     value = ws * st.kv_bytes / (ms_step * 1e-3) / 1e9

@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
                 x[e] = jl <= lim[nt][e] ? s[nt][e] * sl2 : -CUDART_INF_F;
                 x[2 + e] = jh <= lim[nt][e] ? s[nt][2 + e] * sl2 : -CUDART_INF_F;
             }
-            float pr[4];
+            float pr[4], alpha[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 float mx = fmaxf(x[e], x[2 + e]);
@@ -224,19 +224,24 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                 const float m_new = fmaxf(m_run[nt][e], mx);
                 const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
-                const float alpha = fast_exp2(m_run[nt][e] - m_use);
+                alpha[e] = fast_exp2(m_run[nt][e] - m_use);
                 pr[e] = fast_exp2(x[e] - m_use);
                 pr[2 + e] = fast_exp2(x[2 + e] - m_use);
-                l_run[nt][e] = l_run[nt][e] * alpha + pr[e] + pr[2 + e];
                 m_run[nt][e] = m_new;
 #pragma unroll
                 for (int mt = 0; mt < kMT; ++mt) {
-                    acc[nt][mt][e] *= alpha;
-                    acc[nt][mt][2 + e] *= alpha;
+                    acc[nt][mt][e] *= alpha[e];
+                    acc[nt][mt][2 + e] *= alpha[e];
                 }
             }
-            bp[nt][0] = movmatrix_trans(pack_bf16x2(pr[0], pr[1]));
-            bp[nt][1] = movmatrix_trans(pack_bf16x2(pr[2], pr[3]));
+            // P is rounded to bf16 for the PV MMA; the row sums use the same rounded
+            // weights, so the output is an exact convex combination of the V rows
+            const uint32_t w_lo = pack_bf16x2(pr[0], pr[1]), w_hi = pack_bf16x2(pr[2], pr[3]);
+            l_run[nt][0] = l_run[nt][0] * alpha[0] + __uint_as_float(w_lo << 16) + __uint_as_float(w_hi << 16);
+            l_run[nt][1] = l_run[nt][1] * alpha[1] + __uint_as_float(w_lo & 0xffff0000u) +
+                           __uint_as_float(w_hi & 0xffff0000u);
+            bp[nt][0] = movmatrix_trans(w_lo);
+            bp[nt][1] = movmatrix_trans(w_hi);
         }
 
         // ---- O^T[D x 8NT] += V^T . P^T

@@ -317,13 +317,16 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
             for (int ch = 0; ch < kPrefillKeys / 8; ++ch) {
                 float pv[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 8; ++i)
                     pv[i] = fast_exp2(__uint_as_float(sv[ch * 8 + i]) - m_ref);
-                    l_sum += pv[i];
-                }
                 const uint32_t addr = sP + (ch >> 3) * Cfg::kHalfBytes + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
                 const uint32_t w0 = pack_bf16x2(pv[0], pv[1]), w1 = pack_bf16x2(pv[2], pv[3]);
                 const uint32_t w2 = pack_bf16x2(pv[4], pv[5]), w3 = pack_bf16x2(pv[6], pv[7]);
+                // the row sum uses the bf16-rounded weights the PV MMA sees
+                l_sum += (__uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xffff0000u)) +
+                         (__uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xffff0000u)) +
+                         (__uint_as_float(w2 << 16) + __uint_as_float(w2 & 0xffff0000u)) +
+                         (__uint_as_float(w3 << 16) + __uint_as_float(w3 & 0xffff0000u));
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2),
                              "r"(w3)
                              : "memory");

@@ -10,6 +10,10 @@ outputs computed with fp32 accumulation):
     i.e. the error of each head's output vector relative to that vector's
     magnitude (a per-element ratio is meaningless for outputs near zero);
   * lse: max |gpu - oracle| <= 1e-3.
+Where outputs exceed 2.5 in magnitude (stress inputs with V ~ N(3, 1)) bf16's
+own spacing is coarser than 2e-2 (one ulp is 2^-5 in [4, 8)), so the abs gate
+becomes two bf16 half-ulps of the largest output, 2^-7 * max|oracle|; it is
+never looser than that and never tighter than 2e-2.
 """
 from __future__ import annotations
 
@@ -100,7 +104,8 @@ def errors(gpu_out: torch.Tensor, ref: np.ndarray, rows=None) -> dict:
 def assert_parity(gpu_out, ref, gpu_lse=None, ref_lse=None, rows=None, what=""):
     e = errors(gpu_out, ref, rows)
     assert not e["nan"], f"{what}: NaN in GPU output"
-    assert e["max_abs"] <= ATOL, f"{what}: max_abs {e}"
+    atol = max(ATOL, 2.0 ** -7 * float(np.abs(ref).max()) if np.size(ref) else 0.0)
+    assert e["max_abs"] <= atol, f"{what}: max_abs {e} (gate {atol})"
     assert e["max_rel"] <= RTOL, f"{what}: max_rel {e}"
     if gpu_lse is not None and ref_lse is not None:
         gl = gpu_lse.cpu().numpy().astype(np.float64)
