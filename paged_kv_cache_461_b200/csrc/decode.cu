@@ -156,13 +156,15 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
         }
     }
 
-    float m_run[NT][2], l_run[NT][2], acc[NT][kMT][4];
+    // l_run: row sum of the bf16-rounded weights (normalises O); l_ex: exact fp32 sum (for the LSE)
+    float m_run[NT][2], l_run[NT][2], l_ex[NT][2], acc[NT][kMT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             m_run[nt][e] = -CUDART_INF_F;
             l_run[nt][e] = 0.f;
+            l_ex[nt][e] = 0.f;
         }
 #pragma unroll
         for (int mt = 0; mt < kMT; ++mt)
@@ -227,6 +229,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
                 alpha[e] = fast_exp2(m_run[nt][e] - m_use);
                 pr[e] = fast_exp2(x[e] - m_use);
                 pr[2 + e] = fast_exp2(x[2 + e] - m_use);
+                l_ex[nt][e] = l_ex[nt][e] * alpha[e] + pr[e] + pr[2 + e];
                 m_run[nt][e] = m_new;
 #pragma unroll
                 for (int mt = 0; mt < kMT; ++mt) {
@@ -285,17 +288,21 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            float v = l_run[nt][e];
+            float v = l_run[nt][e], w = l_ex[nt][e];
             v += __shfl_xor_sync(0xffffffffu, v, 4);
             v += __shfl_xor_sync(0xffffffffu, v, 8);
             v += __shfl_xor_sync(0xffffffffu, v, 16);
+            w += __shfl_xor_sync(0xffffffffu, w, 4);
+            w += __shfl_xor_sync(0xffffffffu, w, 8);
+            w += __shfl_xor_sync(0xffffffffu, w, 16);
             l_run[nt][e] = v;
+            l_ex[nt][e] = w;
         }
 
     // ---- this warp's state -> its own (now idle) ring
     constexpr int kLd = D + 4; // padded row stride in floats
     float *cbuf = reinterpret_cast<float *>(wbase);
-    float *cml = cbuf + kRows * kLd; // m[kRows], l[kRows]
+    float *cml = cbuf + kRows * kLd; // m[kRows], l_rounded[kRows], l_exact[kRows]
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -314,6 +321,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
                 const int n = nt * 8 + 2 * lane + e;
                 cml[n] = m_run[nt][e];
                 cml[kRows + n] = l_run[nt][e];
+                cml[2 * kRows + n] = l_ex[nt][e];
             }
     }
     __syncthreads();
@@ -332,13 +340,14 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
         M = fmaxf(M, ml[n]);
     }
     float wgt[kDecWarps];
-    float lt = 0.f;
+    float lt = 0.f, lx = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) {
         const float *ml = reinterpret_cast<const float *>(smem + w * kDecStages * Cfg::kStage) + kRows * kLd;
         const float mw = ml[n];
         wgt[w] = (mw == -CUDART_INF_F) ? 0.f : fast_exp2(mw - M);
         lt += ml[kRows + n] * wgt[w];
+        lx += ml[2 * kRows + n] * wgt[w];
     }
     const float inv = lt > 0.f ? 1.f / lt : 0.f;
     float o[kEpt];
@@ -357,7 +366,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
             o[i + 3] += wgt[w] * v.w;
         }
     }
-    const float lse = lt > 0.f ? (M + log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
+    const float lse = lx > 0.f ? (M + log2f(lx)) * 0.69314718055994531f : -CUDART_INF_F;
     const int t = qs + n / p.G;
     const int hq = h * p.G + n % p.G;
     if (n_splits == 1) {

@@ -251,7 +251,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         const int p_row = row < rows ? p_min + row / G : p_max;
         const float sl2 = p.scale_log2;
-        float m_ref = -CUDART_INF_F, l_sum = 0.f;
+        // l_sum: row sum of the bf16-rounded weights (normalises O); l_ex: exact fp32 sum (for the LSE)
+        float m_ref = -CUDART_INF_F, l_sum = 0.f, l_ex = 0.f;
         bool ok = true;
         const bool tail_fix = (L % kBlockSize) != 0 && (p_max / kBlockSize) == ((L - 1) / kBlockSize);
         for (int kt = 0; kt < nkt; ++kt) {
@@ -312,13 +313,16 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
                 tmem_wait_st();
             }
             l_sum *= alpha;
+            l_ex *= alpha;
             // P row -> shared memory, K-major with the 128-byte swizzle: [key half][128 rows][64 keys]
 #pragma unroll
             for (int ch = 0; ch < kPrefillKeys / 8; ++ch) {
                 float pv[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 8; ++i) {
                     pv[i] = fast_exp2(__uint_as_float(sv[ch * 8 + i]) - m_ref);
+                    l_ex += pv[i];
+                }
                 const uint32_t addr = sP + (ch >> 3) * Cfg::kHalfBytes + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
                 const uint32_t w0 = pack_bf16x2(pv[0], pv[1]), w1 = pack_bf16x2(pv[2], pv[3]);
                 const uint32_t w2 = pack_bf16x2(pv[4], pv[5]), w3 = pack_bf16x2(pv[6], pv[7]);
@@ -387,7 +391,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
             }
             if (store && p.lse)
                 p.lse[(int64_t)t * p.Hq + hq] =
-                    l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994531f : -CUDART_INF_F;
+                    l_ex > 0.f ? (m_ref + log2f(l_ex)) * 0.69314718055994531f : -CUDART_INF_F;
         }
     }
 
