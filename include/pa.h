@@ -192,6 +192,45 @@ PA_API pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, con
                                   pa_stream_t stream);
 
 /*
+ * pa_attention_mixed_noalloc -- pa_attention_mixed_ex for callers that cannot
+ * allocate device memory.  (No counterpart in the paper: an addition of this
+ * library.)
+ *
+ * Some callers cannot call cudaMalloc or any allocator at the point where
+ * attention runs: code inside a stream that is being captured by another
+ * framework, a plugin host that owns every allocation, or a runtime whose
+ * memory is fully reserved up front.  This entry point needs no workspace
+ * argument: it uses a scratch array compiled into the library, of
+ * PA_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library
+ * holds until the process exits.  The caller still passes q, the caches, the
+ * metadata, out and lse exactly as for pa_attention_mixed_ex, and the results
+ * are the same.
+ *
+ *  - The first call on a device looks up that device's copy of the array
+ *    (cudaGetSymbolAddress) with the device current; make that first call
+ *    before any stream capture on that device.  Later calls do no CUDA API
+ *    work beyond the launches.
+ *  - Bounds that need more than PA_NOALLOC_SCRATCH_BYTES of workspace
+ *    (pa_workspace_size_ex(...) > PA_NOALLOC_SCRATCH_BYTES) are rejected with
+ *    PA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued; a larger
+ *    kv_split_tokens shrinks the need of long-context decode batches.
+ *  - Every call on a device shares the one array.  Calls whose work can
+ *    overlap on the GPU (different streams, no ordering between them) race on
+ *    it and give undefined results; calls ordered on one stream are safe.
+ *    The array keeps the previous call's contents; each call re-initialises
+ *    everything it reads (status word included) before reading it.
+ *  - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+PA_API pa_status_t pa_attention_mixed_noalloc(const void *q, int32_t num_q_heads, const void *k_cache,
+                                              const void *v_cache, const pa_cache_desc_t *cache,
+                                              const int32_t *query_start_loc, const int32_t *seq_lens,
+                                              const int32_t *block_table, int32_t bt_stride, int32_t num_seqs,
+                                              int32_t num_tokens, int32_t max_query_len, int32_t max_seq_len,
+                                              float softmax_scale, void *out, float *lse,
+                                              const pa_attn_options_t *options, pa_stream_t stream);
+
+/*
  * pa_merge_attn_states -- the split-KV reduce on its own.
  * Given attention states of num_parts disjoint key sets for each (row, head):
  * normalised outputs part_out fp32 [num_rows, num_heads, num_parts, head_dim]

@@ -27,8 +27,9 @@ DEVICE_WAIT_TIMEOUT = 4
 
 # every symbol include/pa.h declares
 EXPORTED = ("pa_abi_version", "pa_status_string", "pa_kv_write", "pa_build_slot_mapping", "pa_workspace_size",
-            "pa_workspace_size_ex", "pa_attention_mixed", "pa_attention_mixed_ex", "pa_merge_attn_states",
-            "pa_debug_gather_kv")
+            "pa_workspace_size_ex", "pa_attention_mixed", "pa_attention_mixed_ex", "pa_attention_mixed_noalloc",
+            "pa_merge_attn_states", "pa_debug_gather_kv")
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class PaError(RuntimeError):
@@ -71,10 +72,11 @@ def lib():
                 ctypes.c_float, _vp, _vp, _vp, _sz]
         L.pa_attention_mixed.argtypes = attn + [_vp]
         L.pa_attention_mixed_ex.argtypes = attn + [ctypes.POINTER(AttnOptions), _vp]
+        L.pa_attention_mixed_noalloc.argtypes = attn[:-2] + [ctypes.POINTER(AttnOptions), _vp]
         L.pa_merge_attn_states.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
         L.pa_debug_gather_kv.argtypes = [_vp, ctypes.POINTER(CacheDesc), _vp, _i32, _vp, _vp]
         for name in ("pa_kv_write", "pa_build_slot_mapping", "pa_attention_mixed", "pa_attention_mixed_ex",
-                     "pa_merge_attn_states", "pa_debug_gather_kv"):
+                     "pa_attention_mixed_noalloc", "pa_merge_attn_states", "pa_debug_gather_kv"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -181,6 +183,31 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
                                        float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(),
                                        ctypes.byref(o) if o else None, _stream(stream)), "pa_attention_mixed")
+    return out
+
+
+def attention_mixed_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                            query_start_loc: torch.Tensor, seq_lens: torch.Tensor, block_table: torch.Tensor,
+                            max_query_len: int, max_seq_len: int, softmax_scale: Optional[float] = None,
+                            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                            kv_split_tokens: int = 0, stream=None) -> torch.Tensor:
+    """pa_attention_mixed_noalloc: like attention_mixed but with the library's built-in scratch
+    (for callers that cannot allocate a workspace; calls that overlap on the GPU race on it)."""
+    _need(q, torch.bfloat16, "q")
+    T, Hq, D = q.shape
+    R = seq_lens.shape[0]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    d = cache_desc(k_cache)
+    o = _opts(kv_split_tokens)
+    _check(lib().pa_attention_mixed_noalloc(_ptr(q), Hq, _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
+                                            _ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
+                                            block_table.stride(0), R, T, int(max_query_len), int(max_seq_len),
+                                            float(softmax_scale), _ptr(out), _ptr(lse),
+                                            ctypes.byref(o) if o else None, _stream(stream)),
+           "pa_attention_mixed_noalloc")
     return out
 
 
