@@ -151,13 +151,21 @@ def _barrier(ws):
 
 
 def _max_over_ranks(x: float, ws: int) -> float:
+    """Slowest rank's value (NCCL on GPUs, gloo on CPU-only process groups)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(bytes_per_rank: float, ms_per_step_local: float, ws: int) -> tuple:
+    """(value, ms_per_step): every rank processes its own replica; the job's step time is the max over ranks."""
+    ms = _max_over_ranks(ms_per_step_local, ws)
+    return ws * bytes_per_rank / (ms * 1e-3) / 1e9, ms
 
 
 # --------------------------------------------------------------------------- our arm
@@ -458,9 +466,7 @@ def main():
     win = []
     ms_total = _time_region(st.step, args.steps, args.warmup, ws, window=win)
     clocks = sampler.stop(*win)
-    ms_total = _max_over_ranks(ms_total, ws)
-    ms_step = ms_total / args.steps
-    value = ws * st.kv_bytes / (ms_step * 1e-3) / 1e9
+    value, ms_step = whole_job_value(st.kv_bytes, ms_total / args.steps, ws)
 
     # dominant kernel roofline: the attention launches (plan + decode + reduce), events on their stream
     att_ms = _attention_only_ms(st, max(20, min(args.steps, 200)))
