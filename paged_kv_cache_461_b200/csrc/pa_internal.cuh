@@ -15,6 +15,7 @@ namespace pa {
 constexpr int kBlockSize = 16;           // tokens per KV block
 constexpr int kDefaultSplitTokens = 1024; // keys per split-KV partition of a decode request
 constexpr int kPrefillRows = 128;        // query rows (tokens x grouped heads) per prefill tile
+constexpr int kPrefillRowsPerCta = 256;  // a prefill work item is a pair of tiles
 constexpr int kPrefillKeys = 128;        // keys per prefill K/V tile (8 blocks)
 
 // Device-visible counters at the start of the workspace (one 256-byte header).

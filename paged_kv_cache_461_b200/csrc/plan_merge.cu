@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p)
                     n_dec = (L + p.split_tokens - 1) / p.split_tokens;
                     red = n_dec > 1 ? 1 : 0;
                 } else {
-                    n_pf = (q_len * p.G + kPrefillRows - 1) / kPrefillRows;
+                    n_pf = (q_len * p.G + kPrefillRowsPerCta - 1) / kPrefillRowsPerCta;
                 }
             }
         }
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p)
         cta_excl_scan3(n_dec, n_pf, red, ed, ep, er, td, tp, tr);
         for (int s = 0; s < n_dec; ++s)
             p.dec_units[carry_dec + ed + s] = make_int2(r, s);
-        for (int k = 0; k < n_pf; ++k) // heaviest (last) q-tile of the request first
+        for (int k = 0; k < n_pf; ++k) // heaviest (last) q-pair of the request first
             p.pf_tiles[carry_pf + ep + k] = make_int2(r, n_pf - 1 - k);
         if (red)
             p.red_list[carry_red + er] = r;

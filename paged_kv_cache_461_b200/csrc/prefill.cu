@@ -1,34 +1,44 @@
 // prefill.cu -- chunked-prefill attention over the paged cache on the 5th-gen
-// tensor cores (tcgen05.mma, accumulators in TMEM).
+// tensor cores (tcgen05.mma, accumulators and P in TMEM).
 //
-// Prefill is compute bound (hn.213312.xyz section 一 "调度器"; shengyayun.com
-// 适用场景).  A chunk of q_len tokens at positions c_r .. c_r+q_len-1 attends
-// causally to its request's cached context plus the chunk itself; chunking
-// must not change the result (hn.213312.xyz section 二.1), which holds here
-// because every row's result depends only on its own position.
+// Prefill is compute bound (hn.213312.xyz section 一, scheduler paragraph;
+// shengyayun.com 适用场景).  A chunk of q_len tokens at positions
+// c_r .. c_r+q_len-1 attends causally to its request's cached context plus the
+// chunk itself; chunking does not change any row's result (hn.213312.xyz
+// section 二.1) because every row depends only on its own position.
 //
-// Work unit = one CTA = (request r, q-tile, kv head h).  A tile is 128 query
-// rows: 128/G tokens x the G query heads that share kv head h (rows ordered
-// token-major), so one K/V tile feeds all heads of the group.
+// Work unit = one CTA = (request r, q-pair, kv head h).  A q-pair is two tiles
+// A and B of 128 query rows each; a tile is 128/G tokens x the G query heads
+// that share kv head h (token-major), so one K/V tile feeds every head of the
+// group and both tiles.
 //
-// Warp roles (192 threads, one CTA per SM):
-//   warp 0      TMA producer: the Q tile once (3-D box {64 d, G heads,
-//               128/G tokens}, 128-byte swizzle), then K and V tiles of 128
-//               keys = 8 paged blocks, each block one 2-D box per 64-column
-//               half, into a 2-stage ring;
-//   warp 1      TMEM allocation (512 columns) and the single MMA-issuing
-//               thread: S_j = Q K_j^T (M=128, N=128, K=head_dim) into one of
-//               two TMEM S buffers, then O += P_{j-1} V_{j-1} (M=128, N=head_dim,
-//               K=16 per paged block) -- S for tile j+1 runs on the tensor core
-//               while the softmax warps work on tile j;
-//   warps 2..5  softmax: thread = query row = TMEM lane; tcgen05.ld its S row,
-//               causal mask by select, running max in the exp2 domain, P as
-//               bf16 into shared memory (128-byte swizzled, K-major) for the
-//               PV MMA; O is rescaled in TMEM only when a row's max grows by
-//               more than 2^8 (otherwise the stale max is kept, which leaves
-//               the normalised result unchanged); epilogue O / l -> bf16.
-// V rows past the end of the sequence in the last block (unused slots) are
-// zeroed in shared memory before the last PV MMA, so 0 * NaN never enters O.
+// Warp roles (320 threads, one CTA per SM):
+//   warp 0      TMA producer: both Q tiles once (3-D boxes {64 d, G heads,
+//               128/G tokens}, 128-byte swizzle), then per 128-key step the K
+//               tile and the V tile (8 paged blocks x 64-column halves, 2-D
+//               boxes) into separate 2-stage rings;
+//   warp 1      TMEM allocation (512 columns: S_A, O_A, S_B, O_B) and the
+//               single MMA-issuing thread.  Order per key step j:
+//                 PV_A(j-1), S_A(j), PV_B(j-1), S_B(j)   (ping-pong)
+//               so the tensor core works on one tile while the other tile's
+//               softmax runs.  S = Q K^T is SS (both operands in smem);
+//               O += P V reads P from TMEM (written over S by the softmax)
+//               and V from smem as an MN-major operand;
+//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: thread =
+//               query row = TMEM lane; tcgen05.ld of its S row, causal mask
+//               by select, row max, P = exp2(s*c - m*c) with packed fp32x2
+//               FMAs, bf16 P back into TMEM over S with tcgen05.st; O is
+//               rescaled in TMEM only when a row's max grows by more than 2^8
+//               (a stale max leaves the normalised result unchanged); the
+//               epilogue writes O / l as bf16.
+// Ordering facts the pipeline relies on: the commit after S_X(j) fires only
+// once every earlier MMA of the issuing thread is done, so when the softmax
+// sees S_X(j) the previous PV_X(j-1) has finished with P_X and O_X; and MMAs
+// issued by one thread run in issue order, so S_X(j) (which overwrites the TMEM
+// columns holding P_X(j-1)) runs after PV_X(j-1) has read them.
+// V rows past the end of the sequence in its last block (unused slots) are
+// zeroed in shared memory by the producer before any PV reads them, so 0 * NaN
+// never enters O.
 #include <math_constants.h>
 
 #include "ptx.cuh"
@@ -40,33 +50,57 @@ namespace {
 template <int D>
 struct PfCfg {
     static constexpr int kHalves = D / 64;
-    static constexpr int kHalfBytes = 128 * 128;        // 128 rows x 128 B
-    static constexpr int kQ = 128 * D * 2;              // Q tile
-    static constexpr int kKV = kPrefillKeys * D * 2;    // one K or V tile (8 blocks)
+    static constexpr int kHalfBytes = 128 * 128;       // 128 rows x 128 B
+    static constexpr int kTile = 128 * D * 2;          // one 128-row Q tile, or one 128-key K or V tile
     static constexpr int kStages = 2;
-    static constexpr int kP = 128 * kPrefillKeys * 2;   // P tile
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQ;
-    static constexpr int kOffV = kOffK + kStages * kKV;
-    static constexpr int kOffP = kOffV + kStages * kKV;
-    static constexpr int kOffBar = kOffP + kP;
+    static constexpr int kOffQ = 0;                    // Q_A, Q_B
+    static constexpr int kOffK = 2 * kTile;            // K ring
+    static constexpr int kOffV = kOffK + kStages * kTile; // V ring
+    static constexpr int kOffBar = kOffV + kStages * kTile;
     static constexpr int kBarBytes = 256;
     static constexpr int kUsed = kOffBar + kBarBytes + 1024;
     // keep one CTA per SM (each CTA allocates all 512 TMEM columns)
     static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
 };
 
-enum PfBar { B_Q = 0, B_KF = 1, B_VF = 3, B_KVE = 5, B_SF = 7, B_SFREE = 9, B_PF = 11, B_PVD = 12, B_FIN = 13, B_NUM = 14 };
+// TMEM columns of the two tiles' S (P aliases its first 64 columns) and O
+__device__ __forceinline__ int col_s(int x) { return x * 256; }
+__device__ __forceinline__ int col_o(int x) { return x * 256 + 128; }
+
+enum PfBar {
+    B_Q = 0,
+    B_KF = 1,    // 2: K stage full
+    B_KE = 3,    // 2: K stage consumed
+    B_VF = 5,    // 2: V stage full
+    B_VE = 7,    // 2: V stage consumed
+    B_SF = 9,    // 2: S_X ready (per tile)
+    B_PF = 11,   // 2: P_X written (per tile, 128 arrivals)
+    B_OF = 13,   // 2: O_X final (per tile)
+    B_VFIX = 15, // V tail zeroed
+    B_FIN = 16,
+    B_NUM = 17
+};
 
 constexpr uint32_t kTmemCols = 512;
-constexpr int kColS = 0;   // two S buffers: columns [0,128) and [128,256)
-constexpr int kColO = 256; // O: columns [256, 256+D)
+constexpr int kThreads = 320;
+
+struct TileGeo {
+    int rows;  // valid query rows (0 = tile absent)
+    int p_min; // position of the first token
+    int p_max; // position of the last token
+    int nkt;   // 128-key steps the tile needs
+};
+
+__device__ __forceinline__ int blocks_in_step(int n_keys, int j)
+{
+    return (min(kPrefillKeys, n_keys - j * kPrefillKeys) + kBlockSize - 1) / kBlockSize;
+}
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                         const __grid_constant__ CUtensorMap tm_k,
-                                                         const __grid_constant__ CUtensorMap tm_v,
-                                                         const AttnParams p)
+__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                              const __grid_constant__ CUtensorMap tm_k,
+                                                              const __grid_constant__ CUtensorMap tm_v,
+                                                              const AttnParams p)
 {
     using Cfg = PfCfg<D>;
     constexpr int kKS = D / 16; // k-steps of Q K^T
@@ -81,29 +115,34 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     const uint32_t sQ = sbase + Cfg::kOffQ;
     const uint32_t sK0 = sbase + Cfg::kOffK;
     const uint32_t sV0 = sbase + Cfg::kOffV;
-    const uint32_t sP = sbase + Cfg::kOffP;
     const uint32_t bar = sbase + Cfg::kOffBar;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffBar + B_NUM * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffBar + B_NUM * 8 + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- tile geometry (same in every thread)
-    const int2 tile = p.pf_tiles[u];
-    const int r = tile.x, qt = tile.y;
+    // ---- geometry of the q-pair (identical in every thread)
+    const int2 work = p.pf_tiles[u];
+    const int r = work.x, qp = work.y;
     const int G = p.G;
-    const int TQ = kPrefillRows / G;
+    const int TQ = kPrefillRows / G; // tokens per 128-row tile
     const int qs = p.qsl[r];
     const int q_len = p.qsl[r + 1] - qs;
     const int L = p.seq_lens[r];
     const int ctx = L - q_len;
-    const int tok0 = qt * TQ;                 // first token of the tile within the request
-    const int n_tok = min(TQ, q_len - tok0);
-    const int rows = n_tok * G;
-    const int p_min = ctx + tok0;             // position of the tile's first token
-    const int p_max = p_min + n_tok - 1;      // position of its last token
-    const int n_keys = p_max + 1;
-    const int nkt = (n_keys + kPrefillKeys - 1) / kPrefillKeys;
+    TileGeo tg[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        const int tok0 = (2 * qp + x) * TQ;
+        const int n_tok = max(0, min(TQ, q_len - tok0));
+        tg[x].rows = n_tok * G;
+        tg[x].p_min = ctx + tok0;
+        tg[x].p_max = ctx + tok0 + n_tok - 1;
+        tg[x].nkt = n_tok ? (tg[x].p_max + kPrefillKeys) / kPrefillKeys : 0;
+    }
+    const int n_steps = max(tg[0].nkt, tg[1].nkt);
+    const int n_keys_all = (tg[1].rows ? tg[1].p_max : tg[0].p_max) + 1; // keys the CTA loads
+    const bool tail_fix = (L % kBlockSize) != 0 && (n_keys_all - 1) / kBlockSize == (L - 1) / kBlockSize;
     const int32_t *bt_row = p.bt + (int64_t)r * p.bt_stride;
 
     // ---- setup: barriers, TMEM
@@ -111,13 +150,14 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         mbar_init(bar + B_Q * 8, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar + (B_KF + s) * 8, 1);
+            mbar_init(bar + (B_KE + s) * 8, 1);
             mbar_init(bar + (B_VF + s) * 8, 1);
-            mbar_init(bar + (B_KVE + s) * 8, 1);
+            mbar_init(bar + (B_VE + s) * 8, 1);
             mbar_init(bar + (B_SF + s) * 8, 1);
-            mbar_init(bar + (B_SFREE + s) * 8, 128);
+            mbar_init(bar + (B_PF + s) * 8, 128);
+            mbar_init(bar + (B_OF + s) * 8, 1);
         }
-        mbar_init(bar + B_PF * 8, 128);
-        mbar_init(bar + B_PVD * 8, 1);
+        mbar_init(bar + B_VFIX * 8, 1);
         mbar_init(bar + B_FIN * 8, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -137,107 +177,160 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     };
 
     if (warp == 0) {
-        // ================= TMA producer
+        // ===================================================== TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(bar + B_Q * 8, Cfg::kQ);
+            const int ntiles = tg[1].rows ? 2 : 1;
+            mbar_arrive_expect_tx(bar + B_Q * 8, ntiles * Cfg::kTile);
+            for (int x = 0; x < ntiles; ++x)
 #pragma unroll
-            for (int hf = 0; hf < Cfg::kHalves; ++hf)
-                tma_load_3d(sQ + hf * Cfg::kHalfBytes, &tm_q, hf * 64, h * G, qs + tok0, bar + B_Q * 8);
+                for (int hf = 0; hf < Cfg::kHalves; ++hf)
+                    tma_load_3d(sQ + x * Cfg::kTile + hf * Cfg::kHalfBytes, &tm_q, hf * 64, h * G,
+                                qs + (2 * qp + x) * TQ, bar + B_Q * 8);
         }
-        int issued = 0;
-        for (int kt = 0; kt < nkt; ++kt) {
-            const int st = kt & 1;
-            if (kt >= 2 && !mbar_wait_warp(bar + (B_KVE + st) * 8, ((kt - 2) >> 1) & 1, abort_flag)) {
-                if (lane == 0)
-                    fail();
-                break;
-            }
-            const int key0 = kt * kPrefillKeys;
-            const int nblk = (min(kPrefillKeys, n_keys - key0) + kBlockSize - 1) / kBlockSize;
-            const uint32_t tx = (uint32_t)(nblk * kBlockSize * D * 2);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar + (B_KF + st) * 8, tx);
-                mbar_arrive_expect_tx(bar + (B_VF + st) * 8, tx);
-            }
-            __syncwarp();
+        bool ok = true;
+        for (int j = 0; j < n_steps; ++j) {
+            const int st = j & 1;
+            const int nblk = blocks_in_step(n_keys_all, j);
+            int y = -kBlockSize; // out-of-bounds box: TMA fills zeros
             if (lane < nblk) {
-                const int bid = bt_row[kt * (kPrefillKeys / kBlockSize) + lane];
-                int y = -kBlockSize;
+                const int bid = bt_row[j * (kPrefillKeys / kBlockSize) + lane];
                 if ((unsigned)bid < (unsigned long long)p.num_blocks)
                     y = (bid * p.Hkv + h) * kBlockSize;
                 else
                     atomicOr(&p.hdr->status, PA_DEVICE_BAD_BLOCK);
+            }
+            const uint32_t tx = (uint32_t)(nblk * kBlockSize * D * 2);
+            // K(j) into stage st once K(j-2) is consumed
+            if (j >= 2 && !mbar_wait_warp(bar + (B_KE + st) * 8, ((j - 2) >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0)
+                mbar_arrive_expect_tx(bar + (B_KF + st) * 8, tx);
+            __syncwarp();
+            if (lane < nblk)
 #pragma unroll
-                for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-                    const uint32_t o = hf * Cfg::kHalfBytes + lane * (kBlockSize * 128);
-                    tma_load_2d(sK0 + st * Cfg::kKV + o, &tm_k, hf * 64, y, bar + (B_KF + st) * 8);
-                    tma_load_2d(sV0 + st * Cfg::kKV + o, &tm_v, hf * 64, y, bar + (B_VF + st) * 8);
+                for (int hf = 0; hf < Cfg::kHalves; ++hf)
+                    tma_load_2d(sK0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128), &tm_k,
+                                hf * 64, y, bar + (B_KF + st) * 8);
+            // V(j) into stage st once V(j-2) is consumed
+            if (j >= 2 && !mbar_wait_warp(bar + (B_VE + st) * 8, ((j - 2) >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0)
+                mbar_arrive_expect_tx(bar + (B_VF + st) * 8, tx);
+            __syncwarp();
+            if (lane < nblk)
+#pragma unroll
+                for (int hf = 0; hf < Cfg::kHalves; ++hf)
+                    tma_load_2d(sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128), &tm_v,
+                                hf * 64, y, bar + (B_VF + st) * 8);
+            if (tail_fix && j == n_steps - 1) {
+                // zero the V rows past the end of the sequence in its last block
+                if (!mbar_wait_warp(bar + (B_VF + st) * 8, (j >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
                 }
+                const int lb = (L - 1) / kBlockSize - j * (kPrefillKeys / kBlockSize);
+                const int first = L % kBlockSize;
+                const int nrow = kBlockSize - first;
+                const int nz = nrow * Cfg::kHalves * 8; // 16-byte chunks
+                for (int i = lane; i < nz; i += 32) {
+                    const int chunk = i & 7;
+                    const int rr = (i >> 3) % nrow;
+                    const int hf = (i >> 3) / nrow;
+                    const uint32_t addr = sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes +
+                                          (lb * kBlockSize + first + rr) * 128 + chunk * 16;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar + B_VFIX * 8);
             }
-            issued = kt + 1;
         }
-        if (*abort_flag && lane == 0) {
-            // let loads already issued land before the CTA exits
-            for (int kt = max(0, issued - 2); kt < issued; ++kt) {
-                (void)mbar_wait(bar + (B_KF + (kt & 1)) * 8, (kt >> 1) & 1);
-                (void)mbar_wait(bar + (B_VF + (kt & 1)) * 8, (kt >> 1) & 1);
-            }
-            (void)mbar_wait(bar + B_Q * 8, 0);
-        }
+        if (!ok && lane == 0)
+            fail();
     } else if (warp == 1) {
-        // ================= MMA issuer (one thread)
+        // ===================================================== MMA issuer (one thread)
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kPrefillKeys, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             bool ok = mbar_wait(bar + B_Q * 8, 0, abort_flag);
-            auto issue_pv = [&](int j) -> bool {
-                const int st = j & 1;
-                if (!mbar_wait(bar + (B_VF + st) * 8, (j >> 1) & 1, abort_flag))
-                    return false;
-                if (!mbar_wait(bar + B_PF * 8, j & 1, abort_flag))
-                    return false;
-                tc_fence_after();
-                const int key0 = j * kPrefillKeys;
-                const int nblk = (min(kPrefillKeys, n_keys - key0) + kBlockSize - 1) / kBlockSize;
-                const uint32_t sV = sV0 + st * Cfg::kKV;
-                for (int kk = 0; kk < nblk; ++kk) {
-                    const uint64_t a = smem_desc_sw128(sP + (kk >> 2) * Cfg::kHalfBytes + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(sV + kk * (kBlockSize * 128), Cfg::kHalfBytes, 1024);
-                    umma_f16(tmem + kColO, a, b, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(bar + (B_KVE + st) * 8);
-                umma_commit(bar + B_PVD * 8);
-                return true;
-            };
-            for (int kt = 0; ok && kt < nkt; ++kt) {
-                const int st = kt & 1;
-                if (!mbar_wait(bar + (B_KF + st) * 8, (kt >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                if (kt >= 2 && !mbar_wait(bar + (B_SFREE + st) * 8, ((kt - 2) >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t sK = sK0 + st * Cfg::kKV;
+            auto issue_s = [&](int x, int j) {
+                const uint32_t sK = sK0 + (j & 1) * Cfg::kTile;
+                const uint32_t q_base = sQ + x * Cfg::kTile;
 #pragma unroll
                 for (int ks = 0; ks < kKS; ++ks) {
                     const uint32_t off = (ks >> 2) * Cfg::kHalfBytes + (ks & 3) * 32;
-                    umma_f16(tmem + kColS + st * kPrefillKeys, smem_desc_sw128(sQ + off, 16, 1024),
+                    umma_f16(tmem + col_s(x), smem_desc_sw128(q_base + off, 16, 1024),
                              smem_desc_sw128(sK + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
                 }
-                umma_commit(bar + (B_SF + st) * 8);
-                if (kt >= 1 && !issue_pv(kt - 1)) {
-                    ok = false;
-                    break;
-                }
-            }
-            if (ok && !issue_pv(nkt - 1))
+                umma_commit(bar + (B_SF + x) * 8);
+            };
+            auto issue_pv = [&](int x, int j) {
+                const uint32_t sV = sV0 + (j & 1) * Cfg::kTile;
+                const int nblk = blocks_in_step(tg[x].p_max + 1, j);
+                for (int kk = 0; kk < nblk; ++kk)
+                    umma_f16_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8,
+                                smem_desc_sw128(sV + kk * (kBlockSize * 128), Cfg::kHalfBytes, 1024), idesc_pv,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            // prologue: S(0) for both tiles
+            if (ok && !mbar_wait(bar + B_KF * 8, 0, abort_flag))
                 ok = false;
+            if (ok) {
+                tc_fence_after();
+                for (int x = 0; x < 2; ++x)
+                    if (tg[x].nkt > 0)
+                        issue_s(x, 0);
+                umma_commit(bar + B_KE * 8); // K(0) consumed
+            }
+            for (int j = 0; ok && j < n_steps; ++j) {
+                const int st = j & 1;
+                bool v_ready = false, k_ready = false;
+                for (int x = 0; x < 2; ++x) {
+                    if (j >= tg[x].nkt)
+                        continue;
+                    if (!mbar_wait(bar + (B_PF + x) * 8, j & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!v_ready) {
+                        const bool fix = tail_fix && j == n_steps - 1;
+                        if (!mbar_wait(bar + (fix ? B_VFIX : (B_VF + st)) * 8, fix ? 0u : (uint32_t)((j >> 1) & 1),
+                                       abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        v_ready = true;
+                    }
+                    tc_fence_after();
+                    issue_pv(x, j);
+                    if (j + 1 < tg[x].nkt) {
+                        if (!k_ready) {
+                            if (!mbar_wait(bar + (B_KF + (st ^ 1)) * 8, ((j + 1) >> 1) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            k_ready = true;
+                            tc_fence_after();
+                        }
+                        issue_s(x, j + 1);
+                    } else {
+                        umma_commit(bar + (B_OF + x) * 8);
+                    }
+                }
+                if (!ok)
+                    break;
+                umma_commit(bar + (B_VE + st) * 8); // V(j) consumed
+                if (j + 1 < n_steps)
+                    umma_commit(bar + (B_KE + (st ^ 1)) * 8); // K(j+1) consumed
+            }
             if (!ok)
                 fail();
             // drain: nothing of ours may still be running on the tensor core at dealloc
@@ -245,153 +338,141 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
             (void)mbar_wait(bar + B_FIN * 8, 0);
         }
     } else {
-        // ================= softmax / correction / epilogue (warps 2..5)
-        const int quad = warp & 3;                // TMEM lane quadrant this warp may access
-        const int row = quad * 32 + lane;         // query row of the tile = TMEM lane
-        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        const int p_row = row < rows ? p_min + row / G : p_max;
-        const float sl2 = p.scale_log2;
-        // l_sum: row sum of the bf16-rounded weights (normalises O); l_ex: exact fp32 sum (for the LSE)
-        float m_ref = -CUDART_INF_F, l_sum = 0.f, l_ex = 0.f;
-        bool ok = true;
-        const bool tail_fix = (L % kBlockSize) != 0 && (p_max / kBlockSize) == ((L - 1) / kBlockSize);
-        for (int kt = 0; kt < nkt; ++kt) {
-            const int buf = kt & 1;
-            if (!mbar_wait_warp(bar + (B_SF + buf) * 8, (kt >> 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t sv[kPrefillKeys];
-#pragma unroll
-            for (int c = 0; c < kPrefillKeys / 32; ++c) {
-                uint32_t tmp[32];
-                tmem_ld32(tmem + lane_addr + kColS + buf * kPrefillKeys + c * 32, tmp);
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    sv[c * 32 + i] = tmp[i];
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar + (B_SFREE + buf) * 8);
-
-            const int key0 = kt * kPrefillKeys;
-            const bool masked = key0 + kPrefillKeys - 1 > p_min;
-            float mx = -CUDART_INF_F;
-#pragma unroll
-            for (int c = 0; c < kPrefillKeys; ++c) {
-                float x = __uint_as_float(sv[c]) * sl2;
-                if (masked && key0 + c > p_row)
-                    x = -CUDART_INF_F;
-                sv[c] = __float_as_uint(x);
-                mx = fmaxf(mx, x);
-            }
-            float alpha = 1.f;
-            if (kt == 0) {
-                m_ref = mx;
-            } else if (mx > m_ref + 8.f) {
-                alpha = fast_exp2(m_ref - mx);
-                m_ref = mx;
-            }
-            // P buffer is free and O is stable once the previous PV has completed
-            if (kt > 0 && !mbar_wait_warp(bar + B_PVD * 8, (kt - 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
-                tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + lane_addr + kColO + c * 32, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tmem + lane_addr + kColO + c * 32, o);
-                }
-                tmem_wait_st();
-            }
-            l_sum *= alpha;
-            l_ex *= alpha;
-            // P row -> shared memory, K-major with the 128-byte swizzle: [key half][128 rows][64 keys]
-#pragma unroll
-            for (int ch = 0; ch < kPrefillKeys / 8; ++ch) {
-                float pv[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    pv[i] = fast_exp2(__uint_as_float(sv[ch * 8 + i]) - m_ref);
-                    l_ex += pv[i];
-                }
-                const uint32_t addr = sP + (ch >> 3) * Cfg::kHalfBytes + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-                const uint32_t w0 = pack_bf16x2(pv[0], pv[1]), w1 = pack_bf16x2(pv[2], pv[3]);
-                const uint32_t w2 = pack_bf16x2(pv[4], pv[5]), w3 = pack_bf16x2(pv[6], pv[7]);
-                // the row sum uses the bf16-rounded weights the PV MMA sees
-                l_sum += (__uint_as_float(w0 << 16) + __uint_as_float(w0 & 0xffff0000u)) +
-                         (__uint_as_float(w1 << 16) + __uint_as_float(w1 & 0xffff0000u)) +
-                         (__uint_as_float(w2 << 16) + __uint_as_float(w2 & 0xffff0000u)) +
-                         (__uint_as_float(w3 << 16) + __uint_as_float(w3 & 0xffff0000u));
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2),
-                             "r"(w3)
-                             : "memory");
-            }
-            fence_proxy_async_smem();
-            if (kt == nkt - 1 && tail_fix) {
-                // zero V rows past the end of the sequence in the block holding key p_max
-                const int st = kt & 1;
-                if (!mbar_wait_warp(bar + (B_VF + st) * 8, (kt >> 1) & 1, abort_flag)) {
+        // ===================================================== softmax / epilogue (warps 2..5: A, 6..9: B)
+        const int x = (warp - 2) >> 2;
+        const TileGeo g = tg[x];
+        if (g.rows > 0) {
+            const int quad = warp & 3;        // TMEM lane quadrant this warp may access
+            const int row = quad * 32 + lane; // query row of the tile = TMEM lane
+            const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+            const uint32_t tS = tmem + lane_addr + col_s(x);
+            const uint32_t tO = tmem + lane_addr + col_o(x);
+            const int p_row = row < g.rows ? g.p_min + row / G : g.p_max;
+            const float c = p.scale_log2;
+            const float thresh = 8.f / c; // 2^8 growth, in raw score units
+            float m_ref = -CUDART_INF_F;  // reference max, raw score units
+            uint64_t l2 = f2_pack(0.f, 0.f); // exact fp32 row sum, two partial lanes
+            bool ok = true;
+            for (int j = 0; j < g.nkt; ++j) {
+                if (!mbar_wait_warp(bar + (B_SF + x) * 8, j & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const int lb = (p_max / kBlockSize) - kt * (kPrefillKeys / kBlockSize);
-                const int first = L % kBlockSize;
-                const int nz = (kBlockSize - first) * Cfg::kHalves * 8; // 16-byte chunks
-                const uint32_t sV = sV0 + st * Cfg::kKV;
-                for (int i = row; i < nz; i += 128) {
-                    const int chunk = i & 7;
-                    const int rr = (i >> 3) % (kBlockSize - first);
-                    const int hf = (i >> 3) / (kBlockSize - first);
-                    const uint32_t addr = sV + hf * Cfg::kHalfBytes + (lb * kBlockSize + first + rr) * 128 + chunk * 16;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
-                }
-                fence_proxy_async_smem();
-            }
-            tc_fence_before();
-            mbar_arrive(bar + B_PF * 8);
-        }
-        // ---- epilogue: O / l -> bf16
-        if (ok && !mbar_wait_warp(bar + B_PVD * 8, (nkt - 1) & 1, abort_flag))
-            ok = false;
-        if (!ok) {
-            if (lane == 0)
-                fail();
-        } else {
-            tc_fence_after();
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-            const bool store = row < rows;
-            const int t = qs + tok0 + row / G;
-            const int hq = h * G + row % G;
-            __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tmem + lane_addr + kColO + c * 32, o);
-                tmem_wait_ld();
-                if (store) {
+                tc_fence_after();
+                const int key0 = j * kPrefillKeys;
+                const bool diag = key0 + kPrefillKeys - 1 > g.p_min; // causal mask needed in this step
+                // pass 1: row max over the step's 128 scores (two 32-column chunks per TMEM wait)
+                float mx = -CUDART_INF_F;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
-                        v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-                        v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-                        v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(dst + c * 32 + i) = v;
+                for (int cc = 0; cc < kPrefillKeys / 32; cc += 2) {
+                    uint32_t a[32], b[32];
+                    tmem_ld32(tS + cc * 32, a);
+                    tmem_ld32(tS + cc * 32 + 32, b);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        float a0 = __uint_as_float(a[i]), a1 = __uint_as_float(a[i + 1]);
+                        float b0 = __uint_as_float(b[i]), b1 = __uint_as_float(b[i + 1]);
+                        if (diag) {
+                            const int ka = key0 + cc * 32 + i, kb = ka + 32;
+                            a0 = ka > p_row ? -CUDART_INF_F : a0;
+                            a1 = ka + 1 > p_row ? -CUDART_INF_F : a1;
+                            b0 = kb > p_row ? -CUDART_INF_F : b0;
+                            b1 = kb + 1 > p_row ? -CUDART_INF_F : b1;
+                        }
+                        mx = fmax3(mx, a0, a1);
+                        mx = fmax3(mx, b0, b1);
                     }
                 }
+                float alpha = 1.f;
+                if (j == 0) {
+                    m_ref = mx;
+                } else if (mx > m_ref + thresh) {
+                    alpha = fast_exp2((m_ref - mx) * c);
+                    m_ref = mx;
+                }
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                    // O_X is stable: S_X(j) completing implies PV_X(j-1) completed
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + cc * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(tO + cc * 32, o);
+                    }
+                    l2 = f2_mul(l2, f2_pack(alpha, alpha));
+                }
+                // pass 2: P = exp2(s*c - m*c) -> bf16 pairs -> TMEM columns [0, 64) of S_X.  Chunk cc
+                // writes columns [16cc, 16cc+16), all of which were read by earlier chunks.
+                const uint64_t c2 = f2_pack(c, c);
+                const float nm = -m_ref * c;
+                const uint64_t nm2 = f2_pack(nm, nm);
+#pragma unroll
+                for (int cc = 0; cc < kPrefillKeys / 32; ++cc) {
+                    uint32_t sv[32];
+                    tmem_ld32(tS + cc * 32, sv);
+                    tmem_wait_ld();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float s0 = __uint_as_float(sv[2 * i]), s1 = __uint_as_float(sv[2 * i + 1]);
+                        if (diag) {
+                            const int k0 = key0 + cc * 32 + 2 * i;
+                            s0 = k0 > p_row ? -CUDART_INF_F : s0;
+                            s1 = k0 + 1 > p_row ? -CUDART_INF_F : s1;
+                        }
+                        float e0, e1;
+                        f2_unpack(f2_fma(f2_pack(s0, s1), c2, nm2), e0, e1);
+                        const float p0 = fast_exp2(e0), p1 = fast_exp2(e1);
+                        l2 = f2_add(l2, f2_pack(p0, p1));
+                        w[i] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + cc * 16, w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar + (B_PF + x) * 8);
             }
-            if (store && p.lse)
-                p.lse[(int64_t)t * p.Hq + hq] =
-                    l_ex > 0.f ? (m_ref + log2f(l_ex)) * 0.69314718055994531f : -CUDART_INF_F;
+            // ---- epilogue: O / l -> bf16
+            if (ok && !mbar_wait_warp(bar + (B_OF + x) * 8, 0, abort_flag))
+                ok = false;
+            if (!ok) {
+                if (lane == 0)
+                    fail();
+            } else {
+                tc_fence_after();
+                float la, lb;
+                f2_unpack(l2, la, lb);
+                const float l_sum = la + lb;
+                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const bool store = row < g.rows;
+                const int t = qs + (2 * qp + x) * TQ + row / G;
+                const int hq = h * G + row % G;
+                __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + cc * 32, o);
+                    tmem_wait_ld();
+                    if (store) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+                            v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                            v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+                            v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+                            *reinterpret_cast<uint4 *>(dst + cc * 32 + i) = v;
+                        }
+                    }
+                }
+                if (store && p.lse)
+                    p.lse[(int64_t)t * p.Hq + hq] =
+                        l_sum > 0.f ? (m_ref * c + log2f(l_sum)) * 0.69314718055994531f : -CUDART_INF_F;
+            }
         }
     }
 
@@ -418,7 +499,7 @@ cudaError_t launch_prefill_t(const AttnParams &p, const CUtensorMap &tq, const C
         attr_done[dev] = true;
     }
     const unsigned grid = (unsigned)(grid_tiles * p.Hkv);
-    prefill_kernel<D><<<grid, 192, smem, s>>>(tq, tk, tv, p);
+    prefill_kernel<D><<<grid, kThreads, smem, s>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
