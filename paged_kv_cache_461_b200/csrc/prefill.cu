@@ -12,7 +12,7 @@
 // that share kv head h (token-major), so one K/V tile feeds every head of the
 // group and both tiles.
 //
-// Warp roles (320 threads, one CTA per SM):
+// Warp roles (576 threads, one CTA per SM):
 //   warp 0      TMA producer: both Q tiles once (3-D boxes {64 d, G heads,
 //               128/G tokens}, 128-byte swizzle), then per 128-key step the K
 //               tile and the V tile (8 paged blocks x 64-column halves, 2-D
@@ -24,13 +24,17 @@
 //               softmax runs.  S = Q K^T is SS (both operands in smem);
 //               O += P V reads P from TMEM (written over S by the softmax)
 //               and V from smem as an MN-major operand;
-//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: thread =
-//               query row = TMEM lane; tcgen05.ld of its S row, causal mask
-//               by select, row max, P = exp2(s*c - m*c) with packed fp32x2
-//               FMAs, bf16 P back into TMEM over S with tcgen05.st; O is
-//               rescaled in TMEM only when a row's max grows by more than 2^8
-//               (a stale max leaves the normalised result unchanged); the
-//               epilogue writes O / l as bf16.
+//   warps 2..9  softmax of tile A, warps 10..17 softmax of tile B: each
+//               query row (= TMEM lane) is shared by two threads in two warps
+//               of the same TMEM lane quadrant, one per 64-key half, so a
+//               thread holds its 64 scores in registers after one tcgen05.ld
+//               pass.  Causal mask by select, row max exchanged between the
+//               two halves through shared memory (64-thread named barrier),
+//               P = exp2(s*c - m*c) with packed fp32x2 FMAs, bf16 P back into
+//               TMEM over S with tcgen05.st; O is rescaled in TMEM only when a
+//               row's max grows by more than 2^8 (a stale max leaves the
+//               normalised result unchanged); the epilogue writes O / l as
+//               bf16, each thread half of the head dimension.
 // Ordering facts the pipeline relies on: the commit after S_X(j) fires only
 // once every earlier MMA of the issuing thread is done, so when the softmax
 // sees S_X(j) the previous PV_X(j-1) has finished with P_X and O_X; and MMAs
@@ -58,7 +62,9 @@ struct PfCfg {
     static constexpr int kOffV = kOffK + kStages * kTile; // V ring
     static constexpr int kOffBar = kOffV + kStages * kTile;
     static constexpr int kBarBytes = 256;
-    static constexpr int kUsed = kOffBar + kBarBytes + 1024;
+    static constexpr int kOffX = kOffBar + kBarBytes;   // row-max / row-sum exchange: [tile][parity][half][128] fp32
+    static constexpr int kXBytes = 2 * 2 * 2 * 128 * 4;
+    static constexpr int kUsed = kOffX + kXBytes + 1024;
     // keep one CTA per SM (each CTA allocates all 512 TMEM columns)
     static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
 };
@@ -74,7 +80,7 @@ enum PfBar {
     B_VF = 5,    // 2: V stage full
     B_VE = 7,    // 2: V stage consumed
     B_SF = 9,    // 2: S_X ready (per tile)
-    B_PF = 11,   // 2: P_X written (per tile, 128 arrivals)
+    B_PF = 11,   // 2: P_X written (per tile, 256 arrivals)
     B_OF = 13,   // 2: O_X final (per tile)
     B_VFIX = 15, // V tail zeroed
     B_FIN = 16,
@@ -82,7 +88,8 @@ enum PfBar {
 };
 
 constexpr uint32_t kTmemCols = 512;
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
+constexpr int kSoftmaxThreads = 256; // per tile: 128 rows x 2 halves
 
 struct TileGeo {
     int rows;  // valid query rows (0 = tile absent)
@@ -154,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             mbar_init(bar + (B_VF + s) * 8, 1);
             mbar_init(bar + (B_VE + s) * 8, 1);
             mbar_init(bar + (B_SF + s) * 8, 1);
-            mbar_init(bar + (B_PF + s) * 8, 128);
+            mbar_init(bar + (B_PF + s) * 8, kSoftmaxThreads);
             mbar_init(bar + (B_OF + s) * 8, 1);
         }
         mbar_init(bar + B_VFIX * 8, 1);
@@ -338,20 +345,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             (void)mbar_wait(bar + B_FIN * 8, 0);
         }
     } else {
-        // ===================================================== softmax / epilogue (warps 2..5: A, 6..9: B)
-        const int x = (warp - 2) >> 2;
-        const TileGeo g = tg[x];
+        // ===================================================== softmax / epilogue (warps 2..9: A, 10..17: B)
+        const int x = (warp - 2) >> 3;          // tile
+        const int half = ((warp - 2) >> 2) & 1; // 64-key half of the row (and half of the head dim)
+        const TileGeo g = x ? tg[1] : tg[0];
         if (g.rows > 0) {
             const int quad = warp & 3;        // TMEM lane quadrant this warp may access
             const int row = quad * 32 + lane; // query row of the tile = TMEM lane
             const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
             const uint32_t tS = tmem + lane_addr + col_s(x);
-            const uint32_t tO = tmem + lane_addr + col_o(x);
+            const uint32_t tO = tmem + lane_addr + col_o(x) + half * (D / 2);
+            const int bar_id = 1 + x * 4 + quad; // named barrier of the two warps sharing these rows
+            float *xch = reinterpret_cast<float *>(smem + Cfg::kOffX) + x * (2 * 2 * 128);
             const int p_row = row < g.rows ? g.p_min + row / G : g.p_max;
             const float c = p.scale_log2;
-            const float thresh = 8.f / c; // 2^8 growth, in raw score units
-            float m_ref = -CUDART_INF_F;  // reference max, raw score units
-            uint64_t l2 = f2_pack(0.f, 0.f); // exact fp32 row sum, two partial lanes
+            const float thresh = 8.f / c;      // 2^8 growth, in raw score units
+            float m_ref = -CUDART_INF_F;       // reference max, raw score units (same in both halves)
+            uint64_t l2 = f2_pack(0.f, 0.f);   // exact fp32 partial row sum of this half
             bool ok = true;
             for (int j = 0; j < g.nkt; ++j) {
                 if (!mbar_wait_warp(bar + (B_SF + x) * 8, j & 1, abort_flag)) {
@@ -359,31 +369,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     break;
                 }
                 tc_fence_after();
-                const int key0 = j * kPrefillKeys;
-                const bool diag = key0 + kPrefillKeys - 1 > g.p_min; // causal mask needed in this step
-                // pass 1: row max over the step's 128 scores (two 32-column chunks per TMEM wait)
+                const int key0 = j * kPrefillKeys + half * 64;
+                const bool diag = j * kPrefillKeys + kPrefillKeys - 1 > g.p_min; // causal mask needed
+                uint32_t sv[64];
+                tmem_ld32p(tS + half * 64, sv);
+                tmem_ld32p(tS + half * 64 + 32, sv + 32);
+                tmem_wait_ld();
+                if (diag) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (key0 + i > p_row)
+                            sv[i] = __float_as_uint(-CUDART_INF_F);
+                }
                 float mx = -CUDART_INF_F;
 #pragma unroll
-                for (int cc = 0; cc < kPrefillKeys / 32; cc += 2) {
-                    uint32_t a[32], b[32];
-                    tmem_ld32(tS + cc * 32, a);
-                    tmem_ld32(tS + cc * 32 + 32, b);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        float a0 = __uint_as_float(a[i]), a1 = __uint_as_float(a[i + 1]);
-                        float b0 = __uint_as_float(b[i]), b1 = __uint_as_float(b[i + 1]);
-                        if (diag) {
-                            const int ka = key0 + cc * 32 + i, kb = ka + 32;
-                            a0 = ka > p_row ? -CUDART_INF_F : a0;
-                            a1 = ka + 1 > p_row ? -CUDART_INF_F : a1;
-                            b0 = kb > p_row ? -CUDART_INF_F : b0;
-                            b1 = kb + 1 > p_row ? -CUDART_INF_F : b1;
-                        }
-                        mx = fmax3(mx, a0, a1);
-                        mx = fmax3(mx, b0, b1);
-                    }
-                }
+                for (int i = 0; i < 64; i += 2)
+                    mx = fmax3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+                // combine with the other half of the row (double-buffered by step parity)
+                float *slot = xch + (j & 1) * 256;
+                slot[half * 128 + row] = mx;
+                asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+                mx = fmaxf(mx, slot[(half ^ 1) * 128 + row]);
                 float alpha = 1.f;
                 if (j == 0) {
                     m_ref = mx;
@@ -391,85 +397,85 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     alpha = fast_exp2((m_ref - mx) * c);
                     m_ref = mx;
                 }
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
-                    // O_X is stable: S_X(j) completing implies PV_X(j-1) completed
-#pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + cc * 32, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(tO + cc * 32, o);
-                    }
-                    l2 = f2_mul(l2, f2_pack(alpha, alpha));
-                }
-                // pass 2: P = exp2(s*c - m*c) -> bf16 pairs -> TMEM columns [0, 64) of S_X.  Chunk cc
-                // writes columns [16cc, 16cc+16), all of which were read by earlier chunks.
+                l2 = f2_mul(l2, f2_pack(alpha, alpha));
+                // P = exp2(s*c - m*c) -> bf16 pairs -> TMEM columns [32*half, 32*half + 32) of S_X.
+                // Both halves finished reading S before the barrier above.
                 const uint64_t c2 = f2_pack(c, c);
                 const float nm = -m_ref * c;
                 const uint64_t nm2 = f2_pack(nm, nm);
 #pragma unroll
-                for (int cc = 0; cc < kPrefillKeys / 32; ++cc) {
-                    uint32_t sv[32];
-                    tmem_ld32(tS + cc * 32, sv);
-                    tmem_wait_ld();
-                    uint32_t w[16];
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t w[8];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float s0 = __uint_as_float(sv[2 * i]), s1 = __uint_as_float(sv[2 * i + 1]);
-                        if (diag) {
-                            const int k0 = key0 + cc * 32 + 2 * i;
-                            s0 = k0 > p_row ? -CUDART_INF_F : s0;
-                            s1 = k0 + 1 > p_row ? -CUDART_INF_F : s1;
-                        }
+                    for (int i = 0; i < 8; ++i) {
                         float e0, e1;
-                        f2_unpack(f2_fma(f2_pack(s0, s1), c2, nm2), e0, e1);
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[cc * 16 + 2 * i]),
+                                                 __uint_as_float(sv[cc * 16 + 2 * i + 1])),
+                                         c2, nm2),
+                                  e0, e1);
                         const float p0 = fast_exp2(e0), p1 = fast_exp2(e1);
                         l2 = f2_add(l2, f2_pack(p0, p1));
                         w[i] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st16(tS + cc * 16, w);
+                    tmem_st8(tS + half * 32 + cc * 8, w);
+                }
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                    // O_X is stable (S_X(j) completing implies PV_X(j-1) completed) and PV_X(j)
+                    // cannot start before the arrive below: rescale this thread's half of the row
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[16];
+                        tmem_ld16(tO + cc * 16, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st16(tO + cc * 16, o);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar + (B_PF + x) * 8);
             }
-            // ---- epilogue: O / l -> bf16
+            // ---- epilogue: O / l -> bf16 (this thread: half of the head dim)
             if (ok && !mbar_wait_warp(bar + (B_OF + x) * 8, 0, abort_flag))
                 ok = false;
+            float la, lb;
+            f2_unpack(l2, la, lb);
+            float l_half = la + lb;
+            // full row sum = both halves' partial sums (exchange slot of parity nkt&1 is free)
+            float *slot = xch + (g.nkt & 1) * 256;
+            slot[half * 128 + row] = l_half;
+            asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+            const float l_sum = l_half + slot[(half ^ 1) * 128 + row];
             if (!ok) {
                 if (lane == 0)
                     fail();
             } else {
                 tc_fence_after();
-                float la, lb;
-                f2_unpack(l2, la, lb);
-                const float l_sum = la + lb;
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
                 const bool store = row < g.rows;
                 const int t = qs + (2 * qp + x) * TQ + row / G;
                 const int hq = h * G + row % G;
-                __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D;
+                __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D + half * (D / 2);
 #pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + cc * 32, o);
+                    uint32_t o[16];
+                    tmem_ld16(tO + cc * 16, o);
                     tmem_wait_ld();
                     if (store) {
 #pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
+                        for (int i = 0; i < 16; i += 8) {
                             uint4 v;
                             v.x = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
                             v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
                             v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
                             v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-                            *reinterpret_cast<uint4 *>(dst + cc * 32 + i) = v;
+                            *reinterpret_cast<uint4 *>(dst + cc * 16 + i) = v;
                         }
                     }
                 }
-                if (store && p.lse)
+                if (store && p.lse && half == 0)
                     p.lse[(int64_t)t * p.Hq + hq] =
                         l_sum > 0.f ? (m_ref * c + log2f(l_sum)) * 0.69314718055994531f : -CUDART_INF_F;
             }
