@@ -268,24 +268,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kPrefillKeys, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             bool ok = mbar_wait(bar + B_Q * 8, 0, abort_flag);
+            // Descriptors are built once; per MMA only the 14-bit start-address field moves, by a
+            // constant number of 16-byte units (shared addresses stay below 2^18, so no carry).
+            const uint64_t dq = smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t dk = smem_desc_sw128(sK0, 16, 1024);
+            const uint64_t dv = smem_desc_sw128(sV0, Cfg::kHalfBytes, 1024);
+            const int pmax0 = tg[0].p_max, pmax1 = tg[1].p_max;
             auto issue_s = [&](int x, int j) {
-                const uint32_t sK = sK0 + (j & 1) * Cfg::kTile;
-                const uint32_t q_base = sQ + x * Cfg::kTile;
+                const uint64_t bq = dq + (uint64_t)((x * Cfg::kTile) >> 4);
+                const uint64_t bk = dk + (uint64_t)(((j & 1) * Cfg::kTile) >> 4);
+                const uint32_t d_tmem = tmem + col_s(x);
+                if constexpr (D == 128) {
+                    // k-steps 0..7: +32 B inside a 128-byte swizzle row, +16 KB to the second 64-column half
+                    constexpr uint32_t H = Cfg::kHalfBytes >> 4;
+                    umma_f16_x8_ss<0, 2, 4, 6, H, H + 2, H + 4, H + 6>(d_tmem, bq, bk, idesc_s, 0u);
+                } else {
 #pragma unroll
-                for (int ks = 0; ks < kKS; ++ks) {
-                    const uint32_t off = (ks >> 2) * Cfg::kHalfBytes + (ks & 3) * 32;
-                    umma_f16(tmem + col_s(x), smem_desc_sw128(q_base + off, 16, 1024),
-                             smem_desc_sw128(sK + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < kKS; ++ks) {
+                        const uint64_t off = (uint64_t)(((ks >> 2) * Cfg::kHalfBytes + (ks & 3) * 32) >> 4);
+                        umma_f16(d_tmem, bq + off, bk + off, idesc_s, ks > 0 ? 1u : 0u);
+                    }
                 }
                 umma_commit(bar + (B_SF + x) * 8);
             };
             auto issue_pv = [&](int x, int j) {
-                const uint32_t sV = sV0 + (j & 1) * Cfg::kTile;
-                const int nblk = blocks_in_step(tg[x].p_max + 1, j);
-                for (int kk = 0; kk < nblk; ++kk)
-                    umma_f16_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8,
-                                smem_desc_sw128(sV + kk * (kBlockSize * 128), Cfg::kHalfBytes, 1024), idesc_pv,
-                                (j > 0 || kk > 0) ? 1u : 0u);
+                const uint64_t bv = dv + (uint64_t)(((j & 1) * Cfg::kTile) >> 4);
+                const int nblk = blocks_in_step((x ? pmax1 : pmax0) + 1, j);
+                const uint32_t d_tmem = tmem + col_o(x);
+                const uint32_t a_tmem = tmem + col_s(x);
+                if (nblk == kPrefillKeys / kBlockSize) {
+                    umma_f16_x8_ts<((kBlockSize * 128) >> 4)>(d_tmem, a_tmem, bv, idesc_pv, j > 0 ? 1u : 0u);
+                } else {
+                    for (int kk = 0; kk < nblk; ++kk)
+                        umma_f16_ts(d_tmem, a_tmem + kk * 8, bv + (uint64_t)((kk * kBlockSize * 128) >> 4),
+                                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                }
             };
             // prologue: S(0) for both tiles
             if (ok && !mbar_wait(bar + B_KF * 8, 0, abort_flag))

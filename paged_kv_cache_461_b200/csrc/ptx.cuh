@@ -244,6 +244,67 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// Eight back-to-back kind::f16 MMAs into one accumulator, operands from shared memory:
+// MMA i uses descriptors a + A_OFF(i) and b + B_OF(i) (16-byte units), offsets given as a
+// compile-time table.  The first MMA overwrites D unless accumulate is set; the rest add.
+template <uint32_t A0, uint32_t A1, uint32_t A2, uint32_t A3, uint32_t A4, uint32_t A5, uint32_t A6, uint32_t A7>
+__device__ __forceinline__ void umma_f16_x8_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p0;\n\t.reg .b64 ra, rb;\n\t"
+        "setp.ne.b32 p0, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p0;\n\t"
+        "add.s64 ra, %1, %5;\n\tadd.s64 rb, %2, %5;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t"
+        "add.s64 ra, %1, %6;\n\tadd.s64 rb, %2, %6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t"
+        "add.s64 ra, %1, %7;\n\tadd.s64 rb, %2, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t"
+        "add.s64 ra, %1, %8;\n\tadd.s64 rb, %2, %8;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t"
+        "add.s64 ra, %1, %9;\n\tadd.s64 rb, %2, %9;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t"
+        "add.s64 ra, %1, %10;\n\tadd.s64 rb, %2, %10;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t"
+        "add.s64 ra, %1, %11;\n\tadd.s64 rb, %2, %11;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "n"((uint64_t)A1), "n"((uint64_t)A2),
+          "n"((uint64_t)A3), "n"((uint64_t)A4), "n"((uint64_t)A5), "n"((uint64_t)A6), "n"((uint64_t)A7)
+        : "memory");
+    (void)A0;
+}
+
+// Eight back-to-back kind::f16 MMAs, A from TMEM (columns a_tmem + 8i), B from shared memory
+// (descriptor b + i * B_STEP in 16-byte units).
+template <uint32_t B_STEP>
+__device__ __forceinline__ void umma_f16_x8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                               uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p0;\n\t.reg .b64 rb;\n\t.reg .b32 ra;\n\t"
+        "setp.ne.b32 p0, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+        "add.u32 ra, %1, 8;\n\tadd.s64 rb, %2, %5;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], rb, %3, 1;\n\t"
+        "add.u32 ra, %1, 16;\n\tadd.s64 rb, %2, %6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], rb, %3, 1;\n\t"
+        "add.u32 ra, %1, 24;\n\tadd.s64 rb, %2, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], rb, %3, 1;\n\t"
+        "add.u32 ra, %1, 32;\n\tadd.s64 rb, %2, %8;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], rb, %3, 1;\n\t"
+        "add.u32 ra, %1, 40;\n\tadd.s64 rb, %2, %9;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], rb, %3, 1;\n\t"
+        "add.u32 ra, %1, 48;\n\tadd.s64 rb, %2, %10;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], rb, %3, 1;\n\t"
+        "add.u32 ra, %1, 56;\n\tadd.s64 rb, %2, %11;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], rb, %3, 1;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "n"((uint64_t)B_STEP),
+          "n"((uint64_t)(2 * B_STEP)), "n"((uint64_t)(3 * B_STEP)), "n"((uint64_t)(4 * B_STEP)),
+          "n"((uint64_t)(5 * B_STEP)), "n"((uint64_t)(6 * B_STEP)), "n"((uint64_t)(7 * B_STEP))
+        : "memory");
+}
+
 // arrive on an mbarrier once all tcgen05 ops issued so far by this thread are done
 __device__ __forceinline__ void umma_commit(uint32_t bar)
 {
