@@ -334,7 +334,7 @@ pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, const void
         if (!get_map(q, 3, D, (uint64_t)num_q_heads, (uint64_t)num_tokens, (uint32_t)P.G,
                      (uint32_t)(kPrefillRows / P.G), &tq))
             return PA_ERR_CUDA;
-        e = launch_prefill(p, tq, tk, tv, P.max_pf_tiles, s);
+        e = launch_prefill(p, tq, tk, tv, P.max_pf_tiles, device_sms(), s);
         if (e != cudaSuccess)
             return PA_ERR_CUDA;
     }

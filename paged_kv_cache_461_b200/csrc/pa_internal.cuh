@@ -16,7 +16,6 @@ constexpr int kBlockSize = 16;           // tokens per KV block
 constexpr int kDefaultSplitTokens = 1024; // keys per split-KV partition of a decode request
 constexpr int kPrefillRows = 128;        // query rows (tokens x grouped heads) per prefill tile
 constexpr int kPrefillRowsPerCta = 256;  // a prefill work item is a pair of tiles
-constexpr int kPrefillKeys = 128;        // keys per prefill K/V tile (8 blocks)
 
 // Device-visible counters at the start of the workspace (one 256-byte header).
 struct WsHeader {
@@ -83,6 +82,6 @@ cudaError_t launch_merge_states(const float *part_out, const float *part_lse, co
                                 int num_rows, int num_heads, int num_parts, int D, void *out, float *lse_out,
                                 cudaStream_t s);
 cudaError_t launch_prefill(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                           int64_t grid_tiles, cudaStream_t s);
+                           int64_t grid_tiles, int num_sms, cudaStream_t s);
 
 } // namespace pa

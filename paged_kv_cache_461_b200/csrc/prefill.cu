@@ -7,39 +7,45 @@
 // chunk itself; chunking does not change any row's result (hn.213312.xyz
 // section 二.1) because every row depends only on its own position.
 //
-// Work unit = one CTA = (request r, q-pair, kv head h).  A q-pair is two tiles
-// A and B of 128 query rows each; a tile is 128/G tokens x the G query heads
-// that share kv head h (token-major), so one K/V tile feeds every head of the
-// group and both tiles.
+// Work item = (request r, q-pair, kv head h).  A q-pair is two tiles A and B of
+// 128 query rows each; a tile is 128/G tokens x the G query heads that share
+// kv head h (token-major), so one K/V tile feeds every head of the group and
+// both tiles.  The kernel is persistent: one CTA per SM walks the work list
+// round-robin, and every ring, barrier phase and counter carries over from one
+// item to the next, so the next item's Q load and first QK^T overlap the
+// previous item's last steps and epilogue.
 //
 // Warp roles (576 threads, one CTA per SM):
-//   warp 0      TMA producer: both Q tiles once (3-D boxes {64 d, G heads,
-//               128/G tokens}, 128-byte swizzle), then per 128-key step the K
-//               tile and the V tile (8 paged blocks x 64-column halves, 2-D
-//               boxes) into separate 2-stage rings;
+//   warp 0      TMA producer: per item both Q tiles (3-D boxes {64 d, G heads,
+//               128/G tokens}, 128-byte swizzle) once the previous item's last
+//               QK^T is done, then per 128-key step the K tile and the V tile (8
+//               paged blocks x 64-column halves, 2-D boxes) into separate
+//               2-stage rings;
 //   warp 1      TMEM allocation (512 columns: S_A, O_A, S_B, O_B) and the
-//               single MMA-issuing thread.  Order per key step j:
+//               single MMA-issuing thread, in the order
 //                 PV_A(j-1), S_A(j), PV_B(j-1), S_B(j)   (ping-pong)
 //               so the tensor core works on one tile while the other tile's
 //               softmax runs.  S = Q K^T is SS (both operands in smem);
-//               O += P V reads P from TMEM (written over S by the softmax)
-//               and V from smem as an MN-major operand;
-//   warps 2..9  softmax of tile A, warps 10..17 softmax of tile B: each
-//               query row (= TMEM lane) is shared by two threads in two warps
-//               of the same TMEM lane quadrant, one per 64-key half, so a
-//               thread holds its 64 scores in registers after one tcgen05.ld
-//               pass.  Causal mask by select, row max exchanged between the
-//               two halves through shared memory (64-thread named barrier),
+//               O += P V reads P from TMEM (written over S by the softmax) and V
+//               from smem as an MN-major operand.  Each group of 8 MMAs is
+//               issued from one asm block with prebuilt descriptors;
+//   warps 2..9  softmax of tile A, warps 10..17 softmax of tile B: each query
+//               row (= TMEM lane) is shared by two threads in two warps of the
+//               same TMEM lane quadrant, one per 64-key half, so a thread holds
+//               its 64 scores in registers after one tcgen05.ld pass.  Causal
+//               mask by select, row max exchanged between the two halves
+//               through shared memory (64-thread named barrier),
 //               P = exp2(s*c - m*c) with packed fp32x2 FMAs, bf16 P back into
 //               TMEM over S with tcgen05.st; O is rescaled in TMEM only when a
 //               row's max grows by more than 2^8 (a stale max leaves the
 //               normalised result unchanged); the epilogue writes O / l as
-//               bf16, each thread half of the head dimension.
-// Ordering facts the pipeline relies on: the commit after S_X(j) fires only
-// once every earlier MMA of the issuing thread is done, so when the softmax
-// sees S_X(j) the previous PV_X(j-1) has finished with P_X and O_X; and MMAs
-// issued by one thread run in issue order, so S_X(j) (which overwrites the TMEM
-// columns holding P_X(j-1)) runs after PV_X(j-1) has read them.
+//               bf16, each thread half of the head dimension, then frees O for
+//               the next item.
+// Ordering facts the pipeline relies on: a commit fires only once every
+// earlier MMA of the issuing thread is done, so when the softmax sees S_X(j)
+// the previous PV_X(j-1) has finished with P_X and O_X; and MMAs issued by one
+// thread run in issue order, so S_X(j) (which overwrites the TMEM columns
+// holding P_X(j-1)) runs after PV_X(j-1) has read them.
 // V rows past the end of the sequence in its last block (unused slots) are
 // zeroed in shared memory by the producer before any PV reads them, so 0 * NaN
 // never enters O.
@@ -50,6 +56,9 @@
 
 namespace pa {
 namespace {
+
+constexpr int kStepKeys = 128;                     // keys per step (8 paged blocks)
+constexpr int kStepBlocks = kStepKeys / kBlockSize;
 
 template <int D>
 struct PfCfg {
@@ -62,9 +71,11 @@ struct PfCfg {
     static constexpr int kOffV = kOffK + kStages * kTile; // V ring
     static constexpr int kOffBar = kOffV + kStages * kTile;
     static constexpr int kBarBytes = 256;
-    static constexpr int kOffX = kOffBar + kBarBytes;   // row-max / row-sum exchange: [tile][parity][half][128] fp32
+    static constexpr int kOffX = kOffBar + kBarBytes;  // per-step row-max exchange: [tile][parity][half][128] fp32
     static constexpr int kXBytes = 2 * 2 * 2 * 128 * 4;
-    static constexpr int kUsed = kOffX + kXBytes + 1024;
+    static constexpr int kOffL = kOffX + kXBytes;      // epilogue row-sum exchange: [tile][half][128] fp32
+    static constexpr int kLBytes = 2 * 2 * 128 * 4;
+    static constexpr int kUsed = kOffL + kLBytes + 1024;
     // keep one CTA per SM (each CTA allocates all 512 TMEM columns)
     static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
 };
@@ -74,17 +85,19 @@ __device__ __forceinline__ int col_s(int x) { return x * 256; }
 __device__ __forceinline__ int col_o(int x) { return x * 256 + 128; }
 
 enum PfBar {
-    B_Q = 0,
-    B_KF = 1,    // 2: K stage full
-    B_KE = 3,    // 2: K stage consumed
-    B_VF = 5,    // 2: V stage full
-    B_VE = 7,    // 2: V stage consumed
-    B_SF = 9,    // 2: S_X ready (per tile)
-    B_PF = 11,   // 2: P_X written (per tile, 256 arrivals)
-    B_OF = 13,   // 2: O_X final (per tile)
-    B_VFIX = 15, // V tail zeroed
-    B_FIN = 16,
-    B_NUM = 17
+    B_Q = 0,     // Q tiles of an item loaded
+    B_QE = 1,    // Q tiles of an item consumed by its last QK^T
+    B_KF = 2,    // 2: K stage full
+    B_KE = 4,    // 2: K stage consumed
+    B_VF = 6,    // 2: V stage full
+    B_VE = 8,    // 2: V stage consumed
+    B_SF = 10,   // 2: S_X ready (per tile)
+    B_PF = 12,   // 2: P_X written (per tile, 256 arrivals)
+    B_OF = 14,   // 2: O_X of an item final (per tile)
+    B_OE = 16,   // 2: O_X of an item read by the epilogue (per tile, 256 arrivals)
+    B_VFIX = 18, // V tail of an item zeroed
+    B_FIN = 19,
+    B_NUM = 20
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -98,9 +111,46 @@ struct TileGeo {
     int nkt;   // 128-key steps the tile needs
 };
 
+struct ItemGeo {
+    int r, qp, h, qs, L, tok0; // tok0: first token of tile A within the request
+    TileGeo t0, t1;
+    int n_steps, n_keys_all;
+    bool tail_fix;
+};
+
+__device__ __forceinline__ ItemGeo item_geo(const AttnParams &p, int item)
+{
+    ItemGeo g;
+    const int u = item / p.Hkv;
+    g.h = item - u * p.Hkv;
+    const int2 work = p.pf_tiles[u];
+    g.r = work.x;
+    g.qp = work.y;
+    const int TQ = kPrefillRows / p.G;
+    g.qs = p.qsl[g.r];
+    const int q_len = p.qsl[g.r + 1] - g.qs;
+    g.L = p.seq_lens[g.r];
+    const int ctx = g.L - q_len;
+    g.tok0 = 2 * g.qp * TQ;
+    const int n0 = max(0, min(TQ, q_len - g.tok0));
+    const int n1 = max(0, min(TQ, q_len - g.tok0 - TQ));
+    g.t0.rows = n0 * p.G;
+    g.t0.p_min = ctx + g.tok0;
+    g.t0.p_max = g.t0.p_min + n0 - 1;
+    g.t0.nkt = n0 ? (g.t0.p_max + kStepKeys) / kStepKeys : 0;
+    g.t1.rows = n1 * p.G;
+    g.t1.p_min = ctx + g.tok0 + TQ;
+    g.t1.p_max = g.t1.p_min + n1 - 1;
+    g.t1.nkt = n1 ? (g.t1.p_max + kStepKeys) / kStepKeys : 0;
+    g.n_steps = max(g.t0.nkt, g.t1.nkt);
+    g.n_keys_all = (n1 ? g.t1.p_max : g.t0.p_max) + 1;
+    g.tail_fix = (g.L % kBlockSize) != 0 && (g.n_keys_all - 1) / kBlockSize == (g.L - 1) / kBlockSize;
+    return g;
+}
+
 __device__ __forceinline__ int blocks_in_step(int n_keys, int j)
 {
-    return (min(kPrefillKeys, n_keys - j * kPrefillKeys) + kBlockSize - 1) / kBlockSize;
+    return (min(kStepKeys, n_keys - j * kStepKeys) + kBlockSize - 1) / kBlockSize;
 }
 
 template <int D>
@@ -111,10 +161,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 {
     using Cfg = PfCfg<D>;
     constexpr int kKS = D / 16; // k-steps of Q K^T
-    const int u = (int)(blockIdx.x / (unsigned)p.Hkv);
-    const int h = (int)(blockIdx.x % (unsigned)p.Hkv);
-    if (u >= (int)p.hdr->n_pf_tiles || (p.hdr->status & PA_DEVICE_WAIT_TIMEOUT))
-        return; // past the work list, or an earlier CTA of this call already gave up
+    const int n_items = (int)p.hdr->n_pf_tiles * p.Hkv;
+    if ((int)blockIdx.x >= n_items || (p.hdr->status & PA_DEVICE_WAIT_TIMEOUT))
+        return; // no work for this CTA, or an earlier CTA of this call already gave up
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -127,34 +176,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffBar + B_NUM * 8 + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // ---- geometry of the q-pair (identical in every thread)
-    const int2 work = p.pf_tiles[u];
-    const int r = work.x, qp = work.y;
     const int G = p.G;
     const int TQ = kPrefillRows / G; // tokens per 128-row tile
-    const int qs = p.qsl[r];
-    const int q_len = p.qsl[r + 1] - qs;
-    const int L = p.seq_lens[r];
-    const int ctx = L - q_len;
-    TileGeo tg[2];
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-        const int tok0 = (2 * qp + x) * TQ;
-        const int n_tok = max(0, min(TQ, q_len - tok0));
-        tg[x].rows = n_tok * G;
-        tg[x].p_min = ctx + tok0;
-        tg[x].p_max = ctx + tok0 + n_tok - 1;
-        tg[x].nkt = n_tok ? (tg[x].p_max + kPrefillKeys) / kPrefillKeys : 0;
-    }
-    const int n_steps = max(tg[0].nkt, tg[1].nkt);
-    const int n_keys_all = (tg[1].rows ? tg[1].p_max : tg[0].p_max) + 1; // keys the CTA loads
-    const bool tail_fix = (L % kBlockSize) != 0 && (n_keys_all - 1) / kBlockSize == (L - 1) / kBlockSize;
-    const int32_t *bt_row = p.bt + (int64_t)r * p.bt_stride;
 
     // ---- setup: barriers, TMEM
     if (threadIdx.x == 0) {
         mbar_init(bar + B_Q * 8, 1);
+        mbar_init(bar + B_QE * 8, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar + (B_KF + s) * 8, 1);
             mbar_init(bar + (B_KE + s) * 8, 1);
@@ -163,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             mbar_init(bar + (B_SF + s) * 8, 1);
             mbar_init(bar + (B_PF + s) * 8, kSoftmaxThreads);
             mbar_init(bar + (B_OF + s) * 8, 1);
+            mbar_init(bar + (B_OE + s) * 8, kSoftmaxThreads);
         }
         mbar_init(bar + B_VFIX * 8, 1);
         mbar_init(bar + B_FIN * 8, 1);
@@ -189,75 +218,90 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            const int ntiles = tg[1].rows ? 2 : 1;
-            mbar_arrive_expect_tx(bar + B_Q * 8, ntiles * Cfg::kTile);
-            for (int x = 0; x < ntiles; ++x)
-#pragma unroll
-                for (int hf = 0; hf < Cfg::kHalves; ++hf)
-                    tma_load_3d(sQ + x * Cfg::kTile + hf * Cfg::kHalfBytes, &tm_q, hf * 64, h * G,
-                                qs + (2 * qp + x) * TQ, bar + B_Q * 8);
         }
         bool ok = true;
-        for (int j = 0; j < n_steps; ++j) {
-            const int st = j & 1;
-            const int nblk = blocks_in_step(n_keys_all, j);
-            int y = -kBlockSize; // out-of-bounds box: TMA fills zeros
-            if (lane < nblk) {
-                const int bid = bt_row[j * (kPrefillKeys / kBlockSize) + lane];
-                if ((unsigned)bid < (unsigned long long)p.num_blocks)
-                    y = (bid * p.Hkv + h) * kBlockSize;
-                else
-                    atomicOr(&p.hdr->status, PA_DEVICE_BAD_BLOCK);
-            }
-            const uint32_t tx = (uint32_t)(nblk * kBlockSize * D * 2);
-            // K(j) into stage st once K(j-2) is consumed
-            if (j >= 2 && !mbar_wait_warp(bar + (B_KE + st) * 8, ((j - 2) >> 1) & 1, abort_flag)) {
+        uint32_t gs = 0; // K/V steps loaded so far by this CTA
+        uint32_t nq = 0; // items whose Q was loaded
+        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+            const ItemGeo g = item_geo(p, item);
+            // Q of this item, once the previous item's last QK^T has read the old Q
+            if (nq > 0 && !mbar_wait_warp(bar + B_QE * 8, (nq - 1) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
-            if (lane == 0)
-                mbar_arrive_expect_tx(bar + (B_KF + st) * 8, tx);
-            __syncwarp();
-            if (lane < nblk)
+            if (lane == 0) {
+                const int ntiles = g.t1.rows ? 2 : 1;
+                mbar_arrive_expect_tx(bar + B_Q * 8, ntiles * Cfg::kTile);
+                for (int x = 0; x < ntiles; ++x)
 #pragma unroll
-                for (int hf = 0; hf < Cfg::kHalves; ++hf)
-                    tma_load_2d(sK0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128), &tm_k,
-                                hf * 64, y, bar + (B_KF + st) * 8);
-            // V(j) into stage st once V(j-2) is consumed
-            if (j >= 2 && !mbar_wait_warp(bar + (B_VE + st) * 8, ((j - 2) >> 1) & 1, abort_flag)) {
-                ok = false;
-                break;
+                    for (int hf = 0; hf < Cfg::kHalves; ++hf)
+                        tma_load_3d(sQ + x * Cfg::kTile + hf * Cfg::kHalfBytes, &tm_q, hf * 64, g.h * G,
+                                    g.qs + g.tok0 + x * TQ, bar + B_Q * 8);
             }
-            if (lane == 0)
-                mbar_arrive_expect_tx(bar + (B_VF + st) * 8, tx);
-            __syncwarp();
-            if (lane < nblk)
-#pragma unroll
-                for (int hf = 0; hf < Cfg::kHalves; ++hf)
-                    tma_load_2d(sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128), &tm_v,
-                                hf * 64, y, bar + (B_VF + st) * 8);
-            if (tail_fix && j == n_steps - 1) {
-                // zero the V rows past the end of the sequence in its last block
-                if (!mbar_wait_warp(bar + (B_VF + st) * 8, (j >> 1) & 1, abort_flag)) {
+            ++nq;
+            const int32_t *bt_row = p.bt + (int64_t)g.r * p.bt_stride;
+            for (int j = 0; j < g.n_steps; ++j, ++gs) {
+                const int st = gs & 1;
+                const int nblk = blocks_in_step(g.n_keys_all, j);
+                int y = -kBlockSize; // out-of-bounds box: TMA fills zeros
+                if (lane < nblk) {
+                    const int bid = bt_row[j * kStepBlocks + lane];
+                    if ((unsigned)bid < (unsigned long long)p.num_blocks)
+                        y = (bid * p.Hkv + g.h) * kBlockSize;
+                    else
+                        atomicOr(&p.hdr->status, PA_DEVICE_BAD_BLOCK);
+                }
+                const uint32_t tx = (uint32_t)(nblk * kBlockSize * D * 2);
+                const uint32_t ph_prev = ((gs >> 1) - 1) & 1; // phase of this stage's previous use
+                // K into stage st once the K two steps back is consumed
+                if (gs >= 2 && !mbar_wait_warp(bar + (B_KE + st) * 8, ph_prev, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const int lb = (L - 1) / kBlockSize - j * (kPrefillKeys / kBlockSize);
-                const int first = L % kBlockSize;
-                const int nrow = kBlockSize - first;
-                const int nz = nrow * Cfg::kHalves * 8; // 16-byte chunks
-                for (int i = lane; i < nz; i += 32) {
-                    const int chunk = i & 7;
-                    const int rr = (i >> 3) % nrow;
-                    const int hf = (i >> 3) / nrow;
-                    const uint32_t addr = sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes +
-                                          (lb * kBlockSize + first + rr) * 128 + chunk * 16;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(bar + B_VFIX * 8);
+                    mbar_arrive_expect_tx(bar + (B_KF + st) * 8, tx);
+                __syncwarp();
+                if (lane < nblk)
+#pragma unroll
+                    for (int hf = 0; hf < Cfg::kHalves; ++hf)
+                        tma_load_2d(sK0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128),
+                                    &tm_k, hf * 64, y, bar + (B_KF + st) * 8);
+                // V into stage st once the V two steps back is consumed
+                if (gs >= 2 && !mbar_wait_warp(bar + (B_VE + st) * 8, ph_prev, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0)
+                    mbar_arrive_expect_tx(bar + (B_VF + st) * 8, tx);
+                __syncwarp();
+                if (lane < nblk)
+#pragma unroll
+                    for (int hf = 0; hf < Cfg::kHalves; ++hf)
+                        tma_load_2d(sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128),
+                                    &tm_v, hf * 64, y, bar + (B_VF + st) * 8);
+                if (g.tail_fix && j == g.n_steps - 1) {
+                    // zero the V rows past the end of the sequence in its last block
+                    if (!mbar_wait_warp(bar + (B_VF + st) * 8, (gs >> 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int lb = (g.L - 1) / kBlockSize - j * kStepBlocks;
+                    const int first = g.L % kBlockSize;
+                    const int nrow = kBlockSize - first;
+                    const int nz = nrow * Cfg::kHalves * 8; // 16-byte chunks
+                    for (int i = lane; i < nz; i += 32) {
+                        const int chunk = i & 7;
+                        const int rr = (i >> 3) % nrow;
+                        const int hf = (i >> 3) / nrow;
+                        const uint32_t addr = sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes +
+                                              (lb * kBlockSize + first + rr) * 128 + chunk * 16;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar + B_VFIX * 8);
+                }
             }
         }
         if (!ok && lane == 0)
@@ -265,18 +309,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     } else if (warp == 1) {
         // ===================================================== MMA issuer (one thread)
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, kPrefillKeys, 0, 0);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, kStepKeys, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-            bool ok = mbar_wait(bar + B_Q * 8, 0, abort_flag);
             // Descriptors are built once; per MMA only the 14-bit start-address field moves, by a
             // constant number of 16-byte units (shared addresses stay below 2^18, so no carry).
             const uint64_t dq = smem_desc_sw128(sQ, 16, 1024);
             const uint64_t dk = smem_desc_sw128(sK0, 16, 1024);
             const uint64_t dv = smem_desc_sw128(sV0, Cfg::kHalfBytes, 1024);
-            const int pmax0 = tg[0].p_max, pmax1 = tg[1].p_max;
-            auto issue_s = [&](int x, int j) {
+            auto issue_s = [&](int x, uint32_t gstep) {
                 const uint64_t bq = dq + (uint64_t)((x * Cfg::kTile) >> 4);
-                const uint64_t bk = dk + (uint64_t)(((j & 1) * Cfg::kTile) >> 4);
+                const uint64_t bk = dk + (uint64_t)(((gstep & 1) * Cfg::kTile) >> 4);
                 const uint32_t d_tmem = tmem + col_s(x);
                 if constexpr (D == 128) {
                     // k-steps 0..7: +32 B inside a 128-byte swizzle row, +16 KB to the second 64-column half
@@ -291,12 +333,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 }
                 umma_commit(bar + (B_SF + x) * 8);
             };
-            auto issue_pv = [&](int x, int j) {
-                const uint64_t bv = dv + (uint64_t)(((j & 1) * Cfg::kTile) >> 4);
-                const int nblk = blocks_in_step((x ? pmax1 : pmax0) + 1, j);
+            auto issue_pv = [&](int x, int j, uint32_t gstep, int p_max) {
+                const uint64_t bv = dv + (uint64_t)(((gstep & 1) * Cfg::kTile) >> 4);
+                const int nblk = blocks_in_step(p_max + 1, j);
                 const uint32_t d_tmem = tmem + col_o(x);
                 const uint32_t a_tmem = tmem + col_s(x);
-                if (nblk == kPrefillKeys / kBlockSize) {
+                if (nblk == kStepBlocks) {
                     umma_f16_x8_ts<((kBlockSize * 128) >> 4)>(d_tmem, a_tmem, bv, idesc_pv, j > 0 ? 1u : 0u);
                 } else {
                     for (int kk = 0; kk < nblk; ++kk)
@@ -304,56 +346,88 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                                     idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };
-            // prologue: S(0) for both tiles
-            if (ok && !mbar_wait(bar + B_KF * 8, 0, abort_flag))
-                ok = false;
-            if (ok) {
+            bool ok = true;
+            uint32_t gs = 0;            // K/V steps consumed so far
+            uint32_t nq = 0;            // items started
+            uint32_t nfix = 0;          // items with a zeroed V tail
+            uint32_t tstep[2] = {0, 0}; // steps of tile X so far (phase of B_SF / B_PF)
+            uint32_t titem[2] = {0, 0}; // items with tile X so far (phase of B_OF / B_OE)
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const ItemGeo g = item_geo(p, item);
+                const int nkt[2] = {g.t0.nkt, g.t1.nkt};
+                const int pmax[2] = {g.t0.p_max, g.t1.p_max};
+                if (!mbar_wait(bar + B_Q * 8, nq & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                // prologue: S(0) for both tiles
+                if (!mbar_wait(bar + (B_KF + (gs & 1)) * 8, (gs >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 for (int x = 0; x < 2; ++x)
-                    if (tg[x].nkt > 0)
-                        issue_s(x, 0);
-                umma_commit(bar + B_KE * 8); // K(0) consumed
-            }
-            for (int j = 0; ok && j < n_steps; ++j) {
-                const int st = j & 1;
-                bool v_ready = false, k_ready = false;
-                for (int x = 0; x < 2; ++x) {
-                    if (j >= tg[x].nkt)
-                        continue;
-                    if (!mbar_wait(bar + (B_PF + x) * 8, j & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!v_ready) {
-                        const bool fix = tail_fix && j == n_steps - 1;
-                        if (!mbar_wait(bar + (fix ? B_VFIX : (B_VF + st)) * 8, fix ? 0u : (uint32_t)((j >> 1) & 1),
-                                       abort_flag)) {
+                    if (nkt[x] > 0)
+                        issue_s(x, gs);
+                umma_commit(bar + (B_KE + (gs & 1)) * 8); // K of step 0 consumed
+                for (int j = 0; ok && j < g.n_steps; ++j) {
+                    const uint32_t gj = gs + j;
+                    bool v_ready = false, k_ready = false;
+                    for (int x = 0; x < 2; ++x) {
+                        if (j >= nkt[x])
+                            continue;
+                        if (!mbar_wait(bar + (B_PF + x) * 8, tstep[x] & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
-                        v_ready = true;
-                    }
-                    tc_fence_after();
-                    issue_pv(x, j);
-                    if (j + 1 < tg[x].nkt) {
-                        if (!k_ready) {
-                            if (!mbar_wait(bar + (B_KF + (st ^ 1)) * 8, ((j + 1) >> 1) & 1, abort_flag)) {
+                        // the first PV of an item overwrites O_X: the previous item's epilogue must be done
+                        if (j == 0 && titem[x] > 0 &&
+                            !mbar_wait(bar + (B_OE + x) * 8, (titem[x] - 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!v_ready) {
+                            const bool fix = g.tail_fix && j == g.n_steps - 1;
+                            if (!mbar_wait(bar + (fix ? B_VFIX : (B_VF + (gj & 1))) * 8,
+                                           fix ? (nfix & 1) : ((gj >> 1) & 1), abort_flag)) {
                                 ok = false;
                                 break;
                             }
-                            k_ready = true;
-                            tc_fence_after();
+                            v_ready = true;
                         }
-                        issue_s(x, j + 1);
-                    } else {
-                        umma_commit(bar + (B_OF + x) * 8);
+                        tc_fence_after();
+                        issue_pv(x, j, gj, pmax[x]);
+                        ++tstep[x];
+                        if (j + 1 < nkt[x]) {
+                            if (!k_ready) {
+                                if (!mbar_wait(bar + (B_KF + ((gj + 1) & 1)) * 8, ((gj + 1) >> 1) & 1, abort_flag)) {
+                                    ok = false;
+                                    break;
+                                }
+                                k_ready = true;
+                                tc_fence_after();
+                            }
+                            issue_s(x, gj + 1);
+                        } else {
+                            umma_commit(bar + (B_OF + x) * 8);
+                        }
                     }
+                    if (!ok)
+                        break;
+                    umma_commit(bar + (B_VE + (gj & 1)) * 8); // V of this step consumed
+                    if (j + 1 < g.n_steps)
+                        umma_commit(bar + (B_KE + ((gj + 1) & 1)) * 8); // K of the next step consumed
                 }
                 if (!ok)
                     break;
-                umma_commit(bar + (B_VE + st) * 8); // V(j) consumed
-                if (j + 1 < n_steps)
-                    umma_commit(bar + (B_KE + (st ^ 1)) * 8); // K(j+1) consumed
+                umma_commit(bar + B_QE * 8); // Q of this item consumed
+                if (g.tail_fix)
+                    ++nfix;
+                gs += g.n_steps;
+                ++nq;
+                for (int x = 0; x < 2; ++x)
+                    if (nkt[x] > 0)
+                        ++titem[x];
             }
             if (!ok)
                 fail();
@@ -365,29 +439,34 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         // ===================================================== softmax / epilogue (warps 2..9: A, 10..17: B)
         const int x = (warp - 2) >> 3;          // tile
         const int half = ((warp - 2) >> 2) & 1; // 64-key half of the row (and half of the head dim)
-        const TileGeo g = x ? tg[1] : tg[0];
-        if (g.rows > 0) {
-            const int quad = warp & 3;        // TMEM lane quadrant this warp may access
-            const int row = quad * 32 + lane; // query row of the tile = TMEM lane
-            const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-            const uint32_t tS = tmem + lane_addr + col_s(x);
-            const uint32_t tO = tmem + lane_addr + col_o(x) + half * (D / 2);
-            const int bar_id = 1 + x * 4 + quad; // named barrier of the two warps sharing these rows
-            float *xch = reinterpret_cast<float *>(smem + Cfg::kOffX) + x * (2 * 2 * 128);
+        const int quad = warp & 3;              // TMEM lane quadrant this warp may access
+        const int row = quad * 32 + lane;       // query row of the tile = TMEM lane
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        const uint32_t tS = tmem + lane_addr + col_s(x);
+        const uint32_t tO = tmem + lane_addr + col_o(x) + half * (D / 2);
+        const int bar_id = 1 + x * 4 + quad; // named barrier of the two warps sharing these rows
+        float *xch = reinterpret_cast<float *>(smem + Cfg::kOffX) + x * (2 * 2 * 128);
+        float *lch = reinterpret_cast<float *>(smem + Cfg::kOffL) + x * (2 * 128);
+        const float c = p.scale_log2;
+        const float thresh = 8.f / c; // 2^8 growth, in raw score units
+        bool ok = true;
+        uint32_t tstep = 0, titem = 0;
+        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+            const ItemGeo gi = item_geo(p, item);
+            const TileGeo g = x ? gi.t1 : gi.t0;
+            if (g.rows == 0)
+                continue;
             const int p_row = row < g.rows ? g.p_min + row / G : g.p_max;
-            const float c = p.scale_log2;
-            const float thresh = 8.f / c;      // 2^8 growth, in raw score units
-            float m_ref = -CUDART_INF_F;       // reference max, raw score units (same in both halves)
-            uint64_t l2 = f2_pack(0.f, 0.f);   // exact fp32 partial row sum of this half
-            bool ok = true;
-            for (int j = 0; j < g.nkt; ++j) {
-                if (!mbar_wait_warp(bar + (B_SF + x) * 8, j & 1, abort_flag)) {
+            float m_ref = -CUDART_INF_F;     // reference max, raw score units (same in both halves)
+            uint64_t l2 = f2_pack(0.f, 0.f); // exact fp32 partial row sum of this half
+            for (int j = 0; j < g.nkt; ++j, ++tstep) {
+                if (!mbar_wait_warp(bar + (B_SF + x) * 8, tstep & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int key0 = j * kPrefillKeys + half * 64;
-                const bool diag = j * kPrefillKeys + kPrefillKeys - 1 > g.p_min; // causal mask needed
+                const int key0 = j * kStepKeys + half * 64;
+                const bool diag = j * kStepKeys + kStepKeys - 1 > g.p_min; // causal mask needed
                 uint32_t sv[64];
                 tmem_ld32p(tS + half * 64, sv);
                 tmem_ld32p(tS + half * 64 + 32, sv + 32);
@@ -403,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 for (int i = 0; i < 64; i += 2)
                     mx = fmax3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
                 // combine with the other half of the row (double-buffered by step parity)
-                float *slot = xch + (j & 1) * 256;
+                float *slot = xch + (tstep & 1) * 256;
                 slot[half * 128 + row] = mx;
                 asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
                 mx = fmaxf(mx, slot[(half ^ 1) * 128 + row]);
@@ -454,49 +533,55 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 tc_fence_before();
                 mbar_arrive(bar + (B_PF + x) * 8);
             }
+            if (!ok)
+                break;
             // ---- epilogue: O / l -> bf16 (this thread: half of the head dim)
-            if (ok && !mbar_wait_warp(bar + (B_OF + x) * 8, 0, abort_flag))
+            if (!mbar_wait_warp(bar + (B_OF + x) * 8, titem & 1, abort_flag)) {
                 ok = false;
+                break;
+            }
             float la, lb;
             f2_unpack(l2, la, lb);
-            float l_half = la + lb;
-            // full row sum = both halves' partial sums (exchange slot of parity nkt&1 is free)
-            float *slot = xch + (g.nkt & 1) * 256;
-            slot[half * 128 + row] = l_half;
+            const float l_half = la + lb;
+            // full row sum = both halves' partial sums.  A partner reads this slot right after
+            // the barrier, before its next step's barrier, so the slot is free again by the
+            // next item's epilogue.
+            lch[half * 128 + row] = l_half;
             asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-            const float l_sum = l_half + slot[(half ^ 1) * 128 + row];
-            if (!ok) {
-                if (lane == 0)
-                    fail();
-            } else {
-                tc_fence_after();
-                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-                const bool store = row < g.rows;
-                const int t = qs + (2 * qp + x) * TQ + row / G;
-                const int hq = h * G + row % G;
-                __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D + half * (D / 2);
+            const float l_sum = l_half + lch[(half ^ 1) * 128 + row];
+            tc_fence_after();
+            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            const bool store = row < g.rows;
+            const int t = gi.qs + gi.tok0 + x * TQ + row / G;
+            const int hq = gi.h * G + row % G;
+            __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D + half * (D / 2);
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[16];
-                    tmem_ld16(tO + cc * 16, o);
-                    tmem_wait_ld();
-                    if (store) {
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[16];
+                tmem_ld16(tO + cc * 16, o);
+                tmem_wait_ld();
+                if (store) {
 #pragma unroll
-                        for (int i = 0; i < 16; i += 8) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
-                            v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-                            v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-                            v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-                            *reinterpret_cast<uint4 *>(dst + cc * 16 + i) = v;
-                        }
+                    for (int i = 0; i < 16; i += 8) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+                        v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                        v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+                        v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(dst + cc * 16 + i) = v;
                     }
                 }
-                if (store && p.lse && half == 0)
-                    p.lse[(int64_t)t * p.Hq + hq] =
-                        l_sum > 0.f ? (m_ref * c + log2f(l_sum)) * 0.69314718055994531f : -CUDART_INF_F;
             }
+            // O_X may now be overwritten by the next item's first PV
+            tc_fence_before();
+            mbar_arrive(bar + (B_OE + x) * 8);
+            ++titem;
+            if (store && p.lse && half == 0)
+                p.lse[(int64_t)t * p.Hq + hq] =
+                    l_sum > 0.f ? (m_ref * c + log2f(l_sum)) * 0.69314718055994531f : -CUDART_INF_F;
         }
+        if (!ok && lane == 0)
+            fail();
     }
 
     tc_fence_before();
@@ -509,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
 template <int D>
 cudaError_t launch_prefill_t(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                             int64_t grid_tiles, cudaStream_t s)
+                             int64_t grid_tiles, int num_sms, cudaStream_t s)
 {
     constexpr int smem = PfCfg<D>::kSmem;
     static bool attr_done[64] = {};
@@ -521,7 +606,9 @@ cudaError_t launch_prefill_t(const AttnParams &p, const CUtensorMap &tq, const C
             return e;
         attr_done[dev] = true;
     }
-    const unsigned grid = (unsigned)(grid_tiles * p.Hkv);
+    // persistent: one CTA per SM, never more CTAs than the largest possible number of items
+    const int64_t items = grid_tiles * p.Hkv;
+    const unsigned grid = (unsigned)(items < num_sms ? items : num_sms);
     prefill_kernel<D><<<grid, kThreads, smem, s>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
@@ -529,13 +616,13 @@ cudaError_t launch_prefill_t(const AttnParams &p, const CUtensorMap &tq, const C
 } // namespace
 
 cudaError_t launch_prefill(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                           int64_t grid_tiles, cudaStream_t s)
+                           int64_t grid_tiles, int num_sms, cudaStream_t s)
 {
     if (grid_tiles <= 0)
         return cudaSuccess;
     if (p.D == 128)
-        return launch_prefill_t<128>(p, tq, tk, tv, grid_tiles, s);
-    return launch_prefill_t<64>(p, tq, tk, tv, grid_tiles, s);
+        return launch_prefill_t<128>(p, tq, tk, tv, grid_tiles, num_sms, s);
+    return launch_prefill_t<64>(p, tq, tk, tv, grid_tiles, num_sms, s);
 }
 
 } // namespace pa

@@ -186,6 +186,10 @@ PREFILL_CASES = [
     (128, 64, 8, [0, 250], [17, 40]),
     (128, 16, 16, [48, 0, 0], [100, 16, 2]),
     (128, 128, 1, [7, 0], [3, 2]),
+    # more work items than SMs: each persistent CTA walks several (request, q-pair, kv head) items
+    (128, 32, 8, [300], [2000]),
+    (128, 32, 8, [0, 1000, 50], [1500, 700, 900]),
+    (64, 16, 16, [0, 17], [4096, 33]),
 ]
 
 
