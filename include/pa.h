@@ -74,9 +74,16 @@ typedef struct pa_cache_desc {
 /* Optional knobs of pa_attention_mixed_ex / pa_workspace_size_ex.  A NULL
  * options pointer, or a zero field, takes the default. */
 typedef struct pa_attn_options {
-    int32_t kv_split_tokens; /* keys per split-KV partition of a decode request;
-                                0 = default (1024); else a positive multiple of 16 */
-    int32_t reserved[7];     /* must be zero */
+    int32_t kv_split_tokens;       /* keys per split-KV partition of a decode request;
+                                      0 = default (1024); else a positive multiple of 16 */
+    int32_t decode_max_query_len;  /* requests with q_len <= this take the memory-bound decode
+                                      kernel instead of the tensor-core prefill kernel, e.g. k+1
+                                      for speculative verification of k drafted tokens
+                                      (shengyayun.com 关键实现细节 3: the target model checks the
+                                      k candidates in one pass); 0 = default (8 / G query rows,
+                                      at least 1).  Allowed up to 16 / G (G = num_q_heads /
+                                      num_kv_heads), else PA_ERR_UNSUPPORTED. */
+    int32_t reserved[6];           /* must be zero */
 } pa_attn_options_t;
 
 /* Bits of the device status word (uint32 at byte 0 of the workspace). */

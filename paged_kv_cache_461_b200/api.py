@@ -44,7 +44,8 @@ class CacheDesc(ctypes.Structure):
 
 
 class AttnOptions(ctypes.Structure):
-    _fields_ = [("kv_split_tokens", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+    _fields_ = [("kv_split_tokens", ctypes.c_int32), ("decode_max_query_len", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
 
 
 _lib = None
@@ -102,11 +103,12 @@ def cache_desc(k_cache: torch.Tensor) -> CacheDesc:
     return CacheDesc(NB, Hkv, D, bs)
 
 
-def _opts(kv_split_tokens: int) -> Optional[AttnOptions]:
-    if not kv_split_tokens:
+def _opts(kv_split_tokens: int, decode_max_query_len: int = 0) -> Optional[AttnOptions]:
+    if not kv_split_tokens and not decode_max_query_len:
         return None
     o = AttnOptions()
     o.kv_split_tokens = int(kv_split_tokens)
+    o.decode_max_query_len = int(decode_max_query_len)
     return o
 
 
@@ -146,15 +148,16 @@ def build_slot_mapping(query_start_loc: torch.Tensor, seq_lens: torch.Tensor, bl
 
 
 def workspace_size(num_seqs: int, num_tokens: int, num_q_heads: int, k_cache_or_desc, max_seq_len: int,
-                   kv_split_tokens: int = 0) -> int:
+                   kv_split_tokens: int = 0, decode_max_query_len: int = 0) -> int:
     d = k_cache_or_desc if isinstance(k_cache_or_desc, CacheDesc) else cache_desc(k_cache_or_desc)
-    o = _opts(kv_split_tokens)
+    o = _opts(kv_split_tokens, decode_max_query_len)
     return int(lib().pa_workspace_size_ex(num_seqs, num_tokens, num_q_heads, ctypes.byref(d), max_seq_len,
                                           ctypes.byref(o) if o else None))
 
 
-def alloc_workspace(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens=0) -> torch.Tensor:
-    n = workspace_size(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens)
+def alloc_workspace(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens=0,
+                    decode_max_query_len=0) -> torch.Tensor:
+    n = workspace_size(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len)
     if n == 0:
         raise PaError(1, "pa_workspace_size")
     return torch.empty(n, dtype=torch.uint8, device=k_cache.device)
@@ -164,7 +167,7 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
                     seq_lens: torch.Tensor, block_table: torch.Tensor, max_query_len: int, max_seq_len: int,
                     softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                     lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                    kv_split_tokens: int = 0, stream=None) -> torch.Tensor:
+                    kv_split_tokens: int = 0, decode_max_query_len: int = 0, stream=None) -> torch.Tensor:
     """pa_attention_mixed[_ex]: q [T, Hq, D] bf16 -> out [T, Hq, D] bf16 (lse [T, Hq] fp32 if given)."""
     _need(q, torch.bfloat16, "q")
     T, Hq, D = q.shape
@@ -174,9 +177,9 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
-        workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens)
+        workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len)
     d = cache_desc(k_cache)
-    o = _opts(kv_split_tokens)
+    o = _opts(kv_split_tokens, decode_max_query_len)
     _check(lib().pa_attention_mixed_ex(_ptr(q), Hq, _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
                                        _ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
                                        block_table.stride(0), R, T, int(max_query_len), int(max_seq_len),

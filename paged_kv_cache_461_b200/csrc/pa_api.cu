@@ -48,7 +48,7 @@ bool make_plan(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, const 
         return false;
     }
     if (o) {
-        for (int i = 0; i < 7; ++i)
+        for (int i = 0; i < 6; ++i)
             if (o->reserved[i] != 0) {
                 *why = PA_ERR_INVALID_ARG;
                 return false;
@@ -63,9 +63,21 @@ bool make_plan(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, const 
         *why = PA_ERR_UNSUPPORTED;
         return false;
     }
-    P.NT = P.G <= 8 ? 1 : (P.G <= 16 ? 2 : 0);
-    P.dec_rows_cap = 8 * P.NT;
-    P.QD = P.NT ? P.dec_rows_cap / P.G : 0;
+    // decode path: up to 8*NT packed (token, head) rows per kv head in one warp MMA
+    const int dq = o ? o->decode_max_query_len : 0;
+    if (dq < 0 || (dq > 0 && dq * P.G > 16)) {
+        *why = dq < 0 ? PA_ERR_INVALID_ARG : PA_ERR_UNSUPPORTED;
+        return false;
+    }
+    if (dq > 0) {
+        P.NT = dq * P.G <= 8 ? 1 : 2;
+        P.QD = dq;
+        P.dec_rows_cap = dq * P.G;
+    } else {
+        P.NT = P.G <= 8 ? 1 : (P.G <= 16 ? 2 : 0);
+        P.dec_rows_cap = 8 * P.NT;
+        P.QD = P.NT ? P.dec_rows_cap / P.G : 0;
+    }
     P.split_tokens = (o && o->kv_split_tokens) ? o->kv_split_tokens : kDefaultSplitTokens;
     const int64_t msl = max_seq_len > 0 ? max_seq_len : 1;
     P.max_splits = P.NT ? (int)((msl + P.split_tokens - 1) / P.split_tokens) : 0;

@@ -69,42 +69,92 @@ __device__ __forceinline__ void cta_excl_scan3(int a, int b, int c, int &ea, int
     __syncthreads();
 }
 
-__global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p)
+// 128-key steps a prefill q-pair of request r needs: keys 0 .. position of its last token
+__device__ __forceinline__ int pair_cost(int ctx, int q_len, int qp, int tq)
 {
+    const int last = min(q_len, (2 * qp + 2) * tq) - 1;
+    return (ctx + last) / 128 + 1;
+}
+
+// Work lists of one step.  Decode units in request order; prefill q-pairs sorted by
+// cost (key steps), most expensive first -- a counting sort through a shared-memory
+// histogram, so the persistent prefill CTAs, which walk the list in snake order, end
+// at nearly the same time.  Pairs of equal cost land in any order; every pair is
+// computed independently, so the order never changes a result.
+__global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_buckets)
+{
+    extern __shared__ int hist[]; // [n_buckets] pair counts, then start offsets
     WsHeader *hdr = p.hdr;
     if (threadIdx.x == 0)
         hdr->status = 0u;
+    for (int i = threadIdx.x; i < n_buckets; i += blockDim.x)
+        hist[i] = 0;
+    __syncthreads();
+    const int tq = kPrefillRows / p.G;
+    auto classify = [&](int r, int &n_dec, int &n_pf, int &red, int &ctx, int &q_len) {
+        n_dec = n_pf = red = 0;
+        ctx = q_len = 0;
+        if (r >= p.num_seqs)
+            return;
+        const int qs = p.qsl[r], qe = p.qsl[r + 1];
+        q_len = qe - qs;
+        const int L = p.seq_lens[r];
+        const bool bad = qs < 0 || qe > p.num_tokens || q_len < 0 || L < q_len || L > p.max_seq_len;
+        if (bad) {
+            atomicOr(&hdr->status, PA_DEVICE_BAD_SEQ);
+            q_len = 0;
+            return;
+        }
+        ctx = L - q_len;
+        if (q_len == 0)
+            return;
+        if (q_len * p.G <= p.dec_rows_cap) {
+            n_dec = (L + p.split_tokens - 1) / p.split_tokens;
+            red = n_dec > 1 ? 1 : 0;
+        } else {
+            n_pf = (q_len * p.G + kPrefillRowsPerCta - 1) / kPrefillRowsPerCta;
+        }
+    };
+    // pass 1: decode units and reduce list in request order; histogram of prefill pair costs
     int carry_dec = 0, carry_pf = 0, carry_red = 0;
     for (int base = 0; base < p.num_seqs; base += blockDim.x) {
         const int r = base + threadIdx.x;
-        int n_dec = 0, n_pf = 0, red = 0;
-        if (r < p.num_seqs) {
-            const int qs = p.qsl[r], qe = p.qsl[r + 1];
-            const int q_len = qe - qs;
-            const int L = p.seq_lens[r];
-            const bool bad = qs < 0 || qe > p.num_tokens || q_len < 0 || L < q_len || L > p.max_seq_len;
-            if (bad) {
-                atomicOr(&hdr->status, PA_DEVICE_BAD_SEQ);
-            } else if (q_len > 0) {
-                if (q_len * p.G <= p.dec_rows_cap) {
-                    n_dec = (L + p.split_tokens - 1) / p.split_tokens;
-                    red = n_dec > 1 ? 1 : 0;
-                } else {
-                    n_pf = (q_len * p.G + kPrefillRowsPerCta - 1) / kPrefillRowsPerCta;
-                }
-            }
-        }
+        int n_dec, n_pf, red, ctx, q_len;
+        classify(r, n_dec, n_pf, red, ctx, q_len);
+        for (int k = 0; k < n_pf; ++k)
+            atomicAdd(&hist[min(pair_cost(ctx, q_len, k, tq), n_buckets - 1)], 1);
         int ed, ep, er, td, tp, tr;
         cta_excl_scan3(n_dec, n_pf, red, ed, ep, er, td, tp, tr);
         for (int s = 0; s < n_dec; ++s)
             p.dec_units[carry_dec + ed + s] = make_int2(r, s);
-        for (int k = 0; k < n_pf; ++k) // heaviest (last) q-pair of the request first
-            p.pf_tiles[carry_pf + ep + k] = make_int2(r, n_pf - 1 - k);
         if (red)
             p.red_list[carry_red + er] = r;
         carry_dec += td;
         carry_pf += tp;
         carry_red += tr;
+    }
+    __syncthreads();
+    // bucket start offsets, most expensive bucket first
+    int carry = 0;
+    for (int base = 0; base < n_buckets; base += blockDim.x) {
+        const int b = n_buckets - 1 - (base + (int)threadIdx.x); // descending cost
+        const int cnt = b >= 0 ? hist[b] : 0;
+        int e0, e1, e2, t0, t1, t2;
+        cta_excl_scan3(cnt, 0, 0, e0, e1, e2, t0, t1, t2);
+        if (b >= 0)
+            hist[b] = carry + e0;
+        carry += t0;
+        __syncthreads();
+    }
+    // pass 2: scatter the prefill pairs into their cost buckets
+    for (int base = 0; base < p.num_seqs; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        int n_dec, n_pf, red, ctx, q_len;
+        classify(r, n_dec, n_pf, red, ctx, q_len);
+        for (int k = 0; k < n_pf; ++k) {
+            const int pos = atomicAdd(&hist[min(pair_cost(ctx, q_len, k, tq), n_buckets - 1)], 1);
+            p.pf_tiles[pos] = make_int2(r, k);
+        }
     }
     if (threadIdx.x == 0) {
         hdr->n_dec_units = (uint32_t)carry_dec;
@@ -217,7 +267,13 @@ __global__ void __launch_bounds__(256) merge_states_kernel(const float *__restri
 
 cudaError_t launch_plan(const AttnParams &p, cudaStream_t s)
 {
-    plan_kernel<<<1, 1024, 0, s>>>(p);
+    // one bucket per possible cost (key steps), capped at 12k buckets (48 KB of shared memory);
+    // costs beyond the last bucket share it
+    int n_buckets = p.max_seq_len / 128 + 2;
+    if (n_buckets > 12 * 1024)
+        n_buckets = 12 * 1024;
+    const int smem = n_buckets * (int)sizeof(int);
+    plan_kernel<<<1, 1024, smem, s>>>(p, n_buckets);
     return cudaGetLastError();
 }
 

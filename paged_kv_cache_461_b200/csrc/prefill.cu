@@ -10,8 +10,8 @@
 // Work item = (request r, q-pair, kv head h).  A q-pair is two tiles A and B of
 // 128 query rows each; a tile is 128/G tokens x the G query heads that share
 // kv head h (token-major), so one K/V tile feeds every head of the group and
-// both tiles.  The kernel is persistent: one CTA per SM walks the work list
-// round-robin, and every ring, barrier phase and counter carries over from one
+// both tiles.  The kernel is persistent: one CTA per SM walks the cost-sorted work
+// list in snake order, and every ring, barrier phase and counter carries over from one
 // item to the next, so the next item's Q load and first QK^T overlap the
 // previous item's last steps and epilogue.
 //
@@ -148,6 +148,15 @@ __device__ __forceinline__ ItemGeo item_geo(const AttnParams &p, int item)
     return g;
 }
 
+// The k-th work item of this CTA.  The work list is sorted by cost, most expensive
+// first; walking it in snake order (CTA b takes item b of even rounds and item
+// grid-1-b of odd rounds) pairs heavy with light items, so the CTAs finish together.
+__device__ __forceinline__ int snake_item(int k)
+{
+    const int b = (k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    return k * (int)gridDim.x + b;
+}
+
 __device__ __forceinline__ int blocks_in_step(int n_keys, int j)
 {
     return (min(kStepKeys, n_keys - j * kStepKeys) + kBlockSize - 1) / kBlockSize;
@@ -222,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         bool ok = true;
         uint32_t gs = 0; // K/V steps loaded so far by this CTA
         uint32_t nq = 0; // items whose Q was loaded
-        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        for (int k = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++k)) {
             const ItemGeo g = item_geo(p, item);
             // Q of this item, once the previous item's last QK^T has read the old Q
             if (nq > 0 && !mbar_wait_warp(bar + B_QE * 8, (nq - 1) & 1, abort_flag)) {
@@ -352,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             uint32_t nfix = 0;          // items with a zeroed V tail
             uint32_t tstep[2] = {0, 0}; // steps of tile X so far (phase of B_SF / B_PF)
             uint32_t titem[2] = {0, 0}; // items with tile X so far (phase of B_OF / B_OE)
-            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+            for (int k = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++k)) {
                 const ItemGeo g = item_geo(p, item);
                 const int nkt[2] = {g.t0.nkt, g.t1.nkt};
                 const int pmax[2] = {g.t0.p_max, g.t1.p_max};
@@ -451,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const float thresh = 8.f / c; // 2^8 growth, in raw score units
         bool ok = true;
         uint32_t tstep = 0, titem = 0;
-        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        for (int k = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++k)) {
             const ItemGeo gi = item_geo(p, item);
             const TileGeo g = x ? gi.t1 : gi.t0;
             if (g.rows == 0)

@@ -62,19 +62,26 @@ class DevStep:
     def write(self):
         api.kv_write(self.k_new, self.v_new, self.slots, self.k_cache, self.v_cache)
 
-    def attend(self, kv_split_tokens=0, with_lse=True, scale=None, workspace=None):
+    def attend(self, kv_split_tokens=0, with_lse=True, scale=None, workspace=None, decode_max_query_len=0):
         lay = self.layout
         lse = torch.full((lay.num_tokens, lay.num_q_heads), float("nan"), dtype=torch.float32,
                          device=self.q.device) if with_lse else None
         out = torch.full_like(self.q, float("nan"))
         if workspace is None:
             workspace = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, self.k_cache,
-                                            lay.max_seq_len, kv_split_tokens)
+                                            lay.max_seq_len, kv_split_tokens, decode_max_query_len)
         api.attention_mixed(self.q, self.k_cache, self.v_cache, self.qsl, self.seq_lens, self.bt,
                             lay.max_query_len, lay.max_seq_len, softmax_scale=scale, out=out, lse=lse,
-                            workspace=workspace, kv_split_tokens=kv_split_tokens)
+                            workspace=workspace, kv_split_tokens=kv_split_tokens,
+                            decode_max_query_len=decode_max_query_len)
         self.workspace = workspace
         return out, lse
+
+
+def work_counts(workspace: torch.Tensor):
+    """(decode units, prefill work items, split requests) the plan kernel wrote into the workspace header."""
+    h = workspace[:16].view(torch.int32).cpu().tolist()
+    return h[1], h[2], h[3]
 
 
 def oracle_for_step(layout: W.StepLayout, vals: W.StepValues, scale=None, token_list=None):

@@ -79,6 +79,14 @@ def test_workspace_size_rules(L):
     assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) > base
     o.reserved[0] = 1
     assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) == 0
+    # decode path for speculative-verify shapes: q_len * G must fit 16 packed rows
+    o = api.AttnOptions()
+    o.decode_max_query_len = 4                      # G = 4: 16 rows
+    assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) > 0
+    o.decode_max_query_len = 5                      # 20 rows
+    assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) == 0
+    o.decode_max_query_len = -1
+    assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) == 0
 
 
 FAKE = 1 << 40  # a non-null pointer value; never dereferenced by host validation paths below

@@ -17,7 +17,8 @@ import torch
 import oracle
 from paged_kv_cache_461_b200 import api, build
 from paged_kv_cache_461_b200 import workloads as W
-from tests.gpu_util import DevStep, assert_parity, bf16_to_f64, errors, oracle_for_step, to_dev_bf16, to_host_bits
+from tests.gpu_util import (DevStep, assert_parity, bf16_to_f64, errors, oracle_for_step, to_dev_bf16, to_host_bits,
+                            work_counts)
 
 pytestmark = pytest.mark.gpu
 
@@ -151,6 +152,35 @@ def test_decode_parity(D, Hq, Hkv, q_len, split):
     st, out, lse, ref, ref_lse = _run(lay, split=split)
     assert_parity(out, ref, lse, ref_lse, what=f"decode D{D} Hq{Hq} Hkv{Hkv} q{q_len} split{split}")
     assert api.read_device_status(st.workspace) == 0
+
+
+SPEC_CASES = [
+    # (Hq, Hkv, q_len = k+1 verified tokens, split): q_len * G packed rows up to 16 in one warp MMA
+    (32, 8, 4, 0), (32, 8, 4, 64), (32, 8, 3, 0), (64, 8, 2, 0), (16, 8, 8, 128), (32, 32, 16, 0),
+]
+
+
+@pytest.mark.parametrize("Hq,Hkv,q_len,split", SPEC_CASES)
+def test_speculative_verify_shapes_take_the_decode_kernel(Hq, Hkv, q_len, split):
+    # the target model scores k drafted tokens plus the last accepted one in a single pass
+    # (shengyayun.com 关键实现细节 3); each verify row attends causally to its own draft prefix
+    rng = np.random.default_rng(Hq + q_len + split)
+    ctx = np.concatenate([rng.integers(20, 900, size=10), [0, 15, 31]])
+    lay = _layout("spec", ctx, np.full(len(ctx), q_len, np.int32), Hq, Hkv, 128, seed=int(ctx.sum()) % 997)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    out, lse = st.attend(kv_split_tokens=split, decode_max_query_len=q_len)
+    torch.cuda.synchronize()
+    n_dec, n_pf, _ = work_counts(st.workspace)
+    assert n_dec > 0 and n_pf == 0, (n_dec, n_pf)
+    ref, ref_lse, _ = oracle_for_step(lay, vals)
+    assert_parity(out, ref, lse, ref_lse, what=f"spec verify Hq{Hq} Hkv{Hkv} q{q_len} split{split}")
+    # the same batch through the prefill kernel agrees within the gate
+    out_pf, _ = st.attend()
+    assert work_counts(st.workspace)[1] > 0 or q_len * Hq // Hkv <= 8
+    e = errors(out, bf16_to_f64(out_pf))
+    assert e["max_abs"] <= 2e-2 and e["max_rel"] <= 1e-2
 
 
 def test_merge_attn_states_matches_oracle_merge():
