@@ -289,7 +289,16 @@ def _prefill_only(st: Step, steps: int, warmup: int):
         call()
     b.record(stream)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps
+    ms = a.elapsed_time(b) / steps
+    # SM clocks under this kernel alone: a back-to-back run of about 0.3 s, sampled by nvidia-smi
+    n = max(steps, int(300.0 / max(ms, 1e-3)))
+    sampler = ClockSampler(torch.cuda.current_device())
+    h0 = time.monotonic()
+    for _ in range(n):
+        call()
+    torch.cuda.synchronize()
+    h1 = time.monotonic()
+    return ms, sampler.stop(h0, h1)
 
 
 def _e2e(st: Step, steps: int, warmup: int):
@@ -496,7 +505,7 @@ def main():
         mx = Step(MIXED)
         mk = max(10, min(args.steps, 100))
         m_ms = _max_over_ranks(_time_region(mx.step, mk, args.warmup, ws), ws) / mk
-        pf_ms = _prefill_only(mx, mk, args.warmup)
+        pf_ms, pf_clocks = _prefill_only(mx, mk, args.warmup)
         pf_tf = mx.prefill_flops / (pf_ms * 1e-3) / 1e12
         line["mixed_step"] = {
             "value": ws * mx.lay.num_tokens / (m_ms * 1e-3), "unit": "tokens/s", "ms_per_step": m_ms,
@@ -505,7 +514,8 @@ def main():
             "prefill_roofline": {"bound": "tensor", "achieved": pf_tf, "peak": peaks["bf16_tflops"],
                                  "unit": "TFLOP/s", "frac": pf_tf / peaks["bf16_tflops"], "ms_per_launch": pf_ms,
                                  "kernel": "pa_attention_mixed on the prefill chunks alone (prefill_kernel)",
-                                 "peak_source": f"{peaks['source']} bf16_tflops (burst)"}}
+                                 "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                                 "clocks": pf_clocks}}
         line["gpu_launches"] += mx.launches_per_step * mk
 
     if rank == 0 and not args.no_cpu_baseline:

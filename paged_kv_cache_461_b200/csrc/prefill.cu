@@ -21,8 +21,8 @@
 //               QK^T is done, then per 128-key step the K tile and the V tile (8
 //               paged blocks x 64-column halves, 2-D boxes) into separate
 //               2-stage rings;
-//   warp 1      TMEM allocation (512 columns: S_A, O_A, S_B, O_B) and the
-//               single MMA-issuing thread, in the order
+//   warp 1      TMEM allocation (512 columns: S_A, O_A, S_B, O_B) and the MMAs
+//               (one elected lane issues, the warp stays converged), in the order
 //                 PV_A(j-1), S_A(j), PV_B(j-1), S_B(j)   (ping-pong)
 //               so the tensor core works on one tile while the other tile's
 //               softmax runs.  S = Q K^T is SS (both operands in smem);
@@ -316,8 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         if (!ok && lane == 0)
             fail();
     } else if (warp == 1) {
-        // ===================================================== MMA issuer (one thread)
-        if (lane == 0) {
+        // ===================================================== MMA issuer (whole warp, one elected lane issues)
+        {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kStepKeys, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             // Descriptors are built once; per MMA only the 14-bit start-address field moves, by a
@@ -365,12 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 const ItemGeo g = item_geo(p, item);
                 const int nkt[2] = {g.t0.nkt, g.t1.nkt};
                 const int pmax[2] = {g.t0.p_max, g.t1.p_max};
-                if (!mbar_wait(bar + B_Q * 8, nq & 1, abort_flag)) {
+                if (!mbar_wait_warp(bar + B_Q * 8, nq & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 // prologue: S(0) for both tiles
-                if (!mbar_wait(bar + (B_KF + (gs & 1)) * 8, (gs >> 1) & 1, abort_flag)) {
+                if (!mbar_wait_warp(bar + (B_KF + (gs & 1)) * 8, (gs >> 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -385,19 +385,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     for (int x = 0; x < 2; ++x) {
                         if (j >= nkt[x])
                             continue;
-                        if (!mbar_wait(bar + (B_PF + x) * 8, tstep[x] & 1, abort_flag)) {
+                        if (!mbar_wait_warp(bar + (B_PF + x) * 8, tstep[x] & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
                         // the first PV of an item overwrites O_X: the previous item's epilogue must be done
                         if (j == 0 && titem[x] > 0 &&
-                            !mbar_wait(bar + (B_OE + x) * 8, (titem[x] - 1) & 1, abort_flag)) {
+                            !mbar_wait_warp(bar + (B_OE + x) * 8, (titem[x] - 1) & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
                         if (!v_ready) {
                             const bool fix = g.tail_fix && j == g.n_steps - 1;
-                            if (!mbar_wait(bar + (fix ? B_VFIX : (B_VF + (gj & 1))) * 8,
+                            if (!mbar_wait_warp(bar + (fix ? B_VFIX : (B_VF + (gj & 1))) * 8,
                                            fix ? (nfix & 1) : ((gj >> 1) & 1), abort_flag)) {
                                 ok = false;
                                 break;
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                         ++tstep[x];
                         if (j + 1 < nkt[x]) {
                             if (!k_ready) {
-                                if (!mbar_wait(bar + (B_KF + ((gj + 1) & 1)) * 8, ((gj + 1) >> 1) & 1, abort_flag)) {
+                                if (!mbar_wait_warp(bar + (B_KF + ((gj + 1) & 1)) * 8, ((gj + 1) >> 1) & 1, abort_flag)) {
                                     ok = false;
                                     break;
                                 }
@@ -438,11 +438,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     if (nkt[x] > 0)
                         ++titem[x];
             }
-            if (!ok)
+            if (!ok && lane == 0)
                 fail();
             // drain: nothing of ours may still be running on the tensor core at dealloc
             umma_commit(bar + B_FIN * 8);
-            (void)mbar_wait(bar + B_FIN * 8, 0);
+            (void)mbar_wait_warp(bar + B_FIN * 8, 0);
         }
     } else {
         // ===================================================== softmax / epilogue (warps 2..9: A, 10..17: B)
