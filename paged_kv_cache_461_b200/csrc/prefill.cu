@@ -381,7 +381,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 umma_commit(bar + (B_KE + (gs & 1)) * 8); // K of step 0 consumed
                 for (int j = 0; ok && j < g.n_steps; ++j) {
                     const uint32_t gj = gs + j;
-                    bool v_ready = false, k_ready = false;
+                    // V of this step (loaded a step earlier, together with the K that S(j) used) and,
+                    // if it has already landed, K of the next step are checked before P: the path from
+                    // a softmax's arrive to its PV issue is then a single barrier wait.
+                    {
+                        const bool fix = g.tail_fix && j == g.n_steps - 1;
+                        if (!mbar_wait_warp(bar + (fix ? B_VFIX : (B_VF + (gj & 1))) * 8,
+                                            fix ? (nfix & 1) : ((gj >> 1) & 1), abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    bool k_ready = j + 1 < g.n_steps &&
+                                   __all_sync(0xffffffffu, mbar_test(bar + (B_KF + ((gj + 1) & 1)) * 8,
+                                                                     ((gj + 1) >> 1) & 1));
                     for (int x = 0; x < 2; ++x) {
                         if (j >= nkt[x])
                             continue;
@@ -394,15 +407,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                             !mbar_wait_warp(bar + (B_OE + x) * 8, (titem[x] - 1) & 1, abort_flag)) {
                             ok = false;
                             break;
-                        }
-                        if (!v_ready) {
-                            const bool fix = g.tail_fix && j == g.n_steps - 1;
-                            if (!mbar_wait_warp(bar + (fix ? B_VFIX : (B_VF + (gj & 1))) * 8,
-                                           fix ? (nfix & 1) : ((gj >> 1) & 1), abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            v_ready = true;
                         }
                         tc_fence_after();
                         issue_pv(x, j, gj, pmax[x]);
@@ -486,10 +490,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                         if (key0 + i > p_row)
                             sv[i] = __float_as_uint(-CUDART_INF_F);
                 }
-                float mx = -CUDART_INF_F;
+                // row max: four independent chains, then combined
+                float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-                for (int i = 0; i < 64; i += 2)
-                    mx = fmax3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+                for (int i = 0; i < 64; i += 8)
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        m4[q4] = fmax3(m4[q4], __uint_as_float(sv[i + 2 * q4]), __uint_as_float(sv[i + 2 * q4 + 1]));
+                float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 // combine with the other half of the row (double-buffered by step parity)
                 float *slot = xch + (tstep & 1) * 256;
                 slot[half * 128 + row] = mx;
@@ -508,22 +516,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 const uint64_t c2 = f2_pack(c, c);
                 const float nm = -m_ref * c;
                 const uint64_t nm2 = f2_pack(nm, nm);
+                uint64_t lb2 = f2_pack(0.f, 0.f); // second row-sum chain
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t w[8];
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t w[16];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
+                    for (int i = 0; i < 16; ++i) {
                         float e0, e1;
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[cc * 16 + 2 * i]),
-                                                 __uint_as_float(sv[cc * 16 + 2 * i + 1])),
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[cc * 32 + 2 * i]),
+                                                 __uint_as_float(sv[cc * 32 + 2 * i + 1])),
                                          c2, nm2),
                                   e0, e1);
                         const float p0 = fast_exp2(e0), p1 = fast_exp2(e1);
-                        l2 = f2_add(l2, f2_pack(p0, p1));
+                        if (i & 1)
+                            lb2 = f2_add(lb2, f2_pack(p0, p1));
+                        else
+                            l2 = f2_add(l2, f2_pack(p0, p1));
                         w[i] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st8(tS + half * 32 + cc * 8, w);
+                    tmem_st16(tS + half * 32 + cc * 16, w);
                 }
+                l2 = f2_add(l2, lb2);
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
                     // O_X is stable (S_X(j) completing implies PV_X(j-1) completed) and PV_X(j)
                     // cannot start before the arrive below: rescale this thread's half of the row
