@@ -337,6 +337,64 @@ def _e2e(st: Step, steps: int, warmup: int):
     return ms, h2d, d2h
 
 
+def _follow_on(st: Step, steps: int, warmup: int, peaks: dict):
+    """The follow-on operations on the headline decode batch: KV write fused into the decode kernel,
+    decode over a token-major (NHD) cache, and whole-block pack / unpack of every block the batch's
+    requests hold.  Events on the launching stream, as for the headline."""
+    import torch
+    api, lay, v = st.api, st.lay, st.vals
+    hbm = peaks["hbm_gbs"]
+    res, launches = {}, 0
+
+    def fused():
+        api.attention_decode_fused(v.q, v.k_new, v.v_new, v.k_cache, v.v_cache, st.qsl, st.seq_lens, st.bt,
+                                   lay.max_query_len, lay.max_seq_len, softmax_scale=st.scale, out=st.out,
+                                   workspace=st.ws)
+    ms_sep = _time_region(st.step, steps, warmup, 1) / steps
+    ms_fused = _time_region(fused, steps, warmup, 1) / steps
+    launches += (2 * st.launches_per_step - 1) * steps
+    res["fused_kv_write_decode"] = {
+        "value": st.kv_bytes / (ms_fused * 1e-3) / 1e9, "unit": "GB/s", "frac": st.kv_bytes / (ms_fused * 1e-3) / 1e9 / hbm,
+        "ms_per_step": ms_fused, "ms_per_step_write_then_attend": ms_sep,
+        "launches_per_step": st.launches_per_step - 1, "launches_per_step_write_then_attend": st.launches_per_step}
+
+    kn, vn = v.k_cache.transpose(1, 2).contiguous(), v.v_cache.transpose(1, 2).contiguous()
+    ws_n = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, kn, lay.max_seq_len, layout="NHD")
+
+    def nhd():
+        api.attention_mixed(v.q, kn, vn, st.qsl, st.seq_lens, st.bt, lay.max_query_len, lay.max_seq_len,
+                            softmax_scale=st.scale, out=st.out, workspace=ws_n, layout="NHD")
+    ms_n = _time_region(nhd, steps, warmup, 1) / steps
+    ms_h = _time_region(st.attention, steps, warmup, 1) / steps
+    launches += 2 * (st.launches_per_step - 1) * steps
+    res["nhd_decode"] = {"value": st.kv_bytes / (ms_n * 1e-3) / 1e9, "unit": "GB/s",
+                         "frac": st.kv_bytes / (ms_n * 1e-3) / 1e9 / hbm, "ms_per_launch": ms_n,
+                         "ms_per_launch_hnd": ms_h, "layout": "[num_blocks, 16, num_kv_heads, head_dim]"}
+    del kn, vn, ws_n
+    torch.cuda.empty_cache()
+
+    nblk = (lay.seq_lens + 15) // 16
+    ids = np.concatenate([lay.block_table[r, :n] for r, n in enumerate(nblk)]).astype(np.int32)
+    ids_d = torch.from_numpy(ids).cuda()
+    elems = lay.num_kv_heads * 16 * lay.head_dim
+    staging = torch.empty((len(ids), 2, elems), dtype=torch.bfloat16, device="cuda")
+    moved = 2 * staging.numel() * 2            # every staged byte is read once and written once
+    ms_pack = _time_region(lambda: api.kv_pack(v.k_cache, v.v_cache, ids_d, staging), steps, warmup, 1) / steps
+    # unpack the staged blocks back over the same blocks (same bytes, same traffic as a fresh pool)
+    ms_unpack = _time_region(lambda: api.kv_unpack(staging, ids_d, v.k_cache, v.v_cache), steps, warmup, 1) / steps
+    launches += 2 * steps
+    res["kv_pack"] = {"value": moved / (ms_pack * 1e-3) / 1e9, "unit": "GB/s",
+                      "frac": moved / (ms_pack * 1e-3) / 1e9 / hbm, "ms_per_launch": ms_pack, "blocks": len(ids),
+                      "bytes_read_plus_written": moved}
+    res["kv_unpack"] = {"value": moved / (ms_unpack * 1e-3) / 1e9, "unit": "GB/s",
+                        "frac": moved / (ms_unpack * 1e-3) / 1e9 / hbm, "ms_per_launch": ms_unpack,
+                        "blocks": len(ids), "bytes_read_plus_written": moved}
+    res["peak"] = {"hbm_gbs": hbm, "source": f"{peaks['source']} hbm_gbs (burst copy)"}
+    del staging
+    torch.cuda.empty_cache()
+    return res, launches
+
+
 # --------------------------------------------------------------------------- CPU oracle leg
 
 def _oracle_sample(name: str, n_requests: int, seed=None):
@@ -499,6 +557,9 @@ def main():
         e_ms, h2d, d2h = _e2e(st, max(10, min(args.steps, 100)), args.warmup)
         line["e2e"] = {"value": st.kv_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    if not args.no_extras and rank == 0:
+        line["follow_on"], n_l = _follow_on(st, max(10, min(args.steps, 50)), args.warmup, peaks)
+        line["gpu_launches"] += n_l
     if not args.no_extras:
         del st
         torch.cuda.empty_cache()

@@ -60,15 +60,23 @@ typedef enum pa_status {
     PA_ERR_CUDA = 4                  /* a CUDA launch or driver call failed */
 } pa_status_t;
 
-/* Both caches have the layout [num_blocks][num_kv_heads][block_size][head_dim]
- * bf16, contiguous: one (block, kv head) is block_size*head_dim*2 bytes
- * (4 KiB at head_dim 128), the unit the kernels fetch.  Slot s is token
- * s % block_size of block s / block_size. */
+/* Layouts of one cache block (the pages fix only the block size, not the
+ * order of the dimensions inside a block). */
+#define PA_LAYOUT_HND 0 /* [num_blocks][num_kv_heads][block_size][head_dim]: one (block, kv head)
+                           is block_size*head_dim*2 contiguous bytes (4 KiB at head_dim 128) */
+#define PA_LAYOUT_NHD 1 /* [num_blocks][block_size][num_kv_heads][head_dim]: one token's rows of
+                           all kv heads are contiguous */
+
+/* K and V caches have the same shape: num_blocks blocks of block_size tokens x
+ * num_kv_heads x head_dim bf16, contiguous, in the given layout.  A whole block
+ * is num_kv_heads*block_size*head_dim*2 contiguous bytes in either layout.
+ * Slot s is token s % block_size of block s / block_size. */
 typedef struct pa_cache_desc {
     int64_t num_blocks;    /* > 0; num_blocks*num_kv_heads*block_size must be < 2^31 */
     int32_t num_kv_heads;  /* > 0 */
     int32_t head_dim;      /* 64 or 128 */
     int32_t block_size;    /* 16 (vLLM's default block size) */
+    int32_t layout;        /* PA_LAYOUT_HND (0) or PA_LAYOUT_NHD (1); anything else is INVALID_ARG */
 } pa_cache_desc_t;
 
 /* Optional knobs of pa_attention_mixed_ex / pa_workspace_size_ex.  A NULL
@@ -92,7 +100,7 @@ typedef struct pa_attn_options {
 #define PA_DEVICE_BAD_BLOCK 2u    /* a block id outside [0, num_blocks) was read (as zeros) */
 #define PA_DEVICE_WAIT_TIMEOUT 4u /* a kernel gave up waiting on a copy or a tensor-core result */
 
-PA_API int32_t pa_abi_version(void); /* 1 */
+PA_API int32_t pa_abi_version(void); /* 2 */
 PA_API const char *pa_status_string(pa_status_t status);
 
 /*
@@ -252,6 +260,65 @@ PA_API pa_status_t pa_attention_mixed_noalloc(const void *q, int32_t num_q_heads
 PA_API pa_status_t pa_merge_attn_states(const float *part_out, const float *part_lse, const int32_t *parts_per_row,
                                  int32_t num_rows, int32_t num_heads, int32_t num_parts, int32_t head_dim,
                                  void *out, float *lse_out, pa_stream_t stream);
+
+/*
+ * pa_attention_decode_fused -- KV write and decode attention of a decode step
+ * in one pass.  (hn.213312.xyz section 一, forward-pass paragraph: each step
+ * writes the new tokens' K/V into their slots, then attends over the cache.)
+ *
+ * Same arguments, rules and results as pa_attention_mixed_ex, plus this
+ * step's new rows k_new/v_new (bf16, token t's row at element
+ * t*new_row_stride, [Hkv, head_dim] contiguous, as for pa_kv_write).  The
+ * new rows of every request -- positions c_r .. L_r-1, slot taken from the
+ * block table as pa_build_slot_mapping does -- are stored into k_cache /
+ * v_cache by the attention kernel itself, which also places them straight
+ * into the tile it attends over instead of reading them back.  The cache
+ * bytes afterwards equal those of pa_kv_write with that slot mapping, and
+ * out / lse are bit-identical to pa_kv_write followed by
+ * pa_attention_mixed_ex.  Requests skipped for bad metadata (device status
+ * bit PA_DEVICE_BAD_SEQ) and rows in a block whose id is outside the pool
+ * are not written.
+ *
+ * Every request must take the decode kernel: max_query_len * G must not
+ * exceed the decode row limit (8 rows per kv head by default, 16 with
+ * options->decode_max_query_len), else PA_ERR_UNSUPPORTED.  k_new, v_new
+ * 16-byte aligned with new_row_stride a multiple of 8, else UNSUPPORTED.
+ * The workspace is sized by pa_workspace_size_ex as for the unfused call.
+ */
+PA_API pa_status_t pa_attention_decode_fused(const void *q, int32_t num_q_heads, const void *k_new,
+                                             const void *v_new, int64_t new_row_stride, void *k_cache,
+                                             void *v_cache, const pa_cache_desc_t *cache,
+                                             const int32_t *query_start_loc, const int32_t *seq_lens,
+                                             const int32_t *block_table, int32_t bt_stride, int32_t num_seqs,
+                                             int32_t num_tokens, int32_t max_query_len, int32_t max_seq_len,
+                                             float softmax_scale, void *out, float *lse, void *workspace,
+                                             size_t workspace_bytes, const pa_attn_options_t *options,
+                                             pa_stream_t stream);
+
+/*
+ * pa_kv_pack / pa_kv_unpack -- copy whole cache blocks to and from a
+ * contiguous staging buffer, e.g. to move a request's KV between a prefill
+ * instance and a decode instance (hn.213312.xyz section 二, item 5, and
+ * shengyayun.com 关键实现细节 item 4: with prefill/decode disaggregation the
+ * prefill side hands its finished KV blocks to the decode side through a
+ * transfer connector).
+ *
+ * staging: bf16 [num_ids][2][block_elems], block_elems =
+ *   num_kv_heads*block_size*head_dim; entry i holds block block_ids[i] of
+ *   k_cache (index 0) then of v_cache (index 1), byte for byte in the cache's
+ *   own layout (a receiver must use the same layout and head_dim).
+ * pack:   staging[i][0] = k_cache block block_ids[i], staging[i][1] = v block;
+ *         an id outside [0, num_blocks) packs zeros.
+ * unpack: the inverse, k_cache block block_ids[i] = staging[i][0] (same for
+ *         V); an id outside the pool is skipped, no other cache byte is
+ *         written.  Duplicate ids in one unpack leave those blocks undefined.
+ * block_ids: device int32 [num_ids].  Every pointer 16-byte aligned, else
+ * PA_ERR_UNSUPPORTED; staging must not overlap the caches.
+ */
+PA_API pa_status_t pa_kv_pack(const void *k_cache, const void *v_cache, const pa_cache_desc_t *cache,
+                              const int32_t *block_ids, int32_t num_ids, void *staging, pa_stream_t stream);
+PA_API pa_status_t pa_kv_unpack(const void *staging, const int32_t *block_ids, int32_t num_ids, void *k_cache,
+                                void *v_cache, const pa_cache_desc_t *cache, pa_stream_t stream);
 
 /*
  * pa_debug_gather_kv -- test helper: contiguous copy of one request's first

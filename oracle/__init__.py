@@ -13,7 +13,8 @@ Parity pins (see tests/test_oracle_*.py): pure-Python brute force, closed
 forms (constant V, zero Q, single key, peaked softmax, a hand-worked two-key
 example), torch's fp64 scaled_dot_product_attention on unpaged data,
 block-id permutation invariance, shared-vs-private prefix blocks, chunked
-prefill invariance, split/merge identity and the KV-write round trip.
+prefill invariance, split/merge identity, the KV-write round trip and the
+block pack/unpack round trip checked against the gather.
 """
 from __future__ import annotations
 
@@ -58,6 +59,10 @@ def _bind(path: str):
     L.oracle_gather_kv.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                    ctypes.c_int32, _i32p, ctypes.c_int64, ctypes.c_int32, _u16p]
     L.oracle_gather_kv.restype = ctypes.c_int
+    L.oracle_kv_pack.argtypes = [_u16p, _u16p, ctypes.c_int64, ctypes.c_int64, _i32p, ctypes.c_int64, _u16p]
+    L.oracle_kv_pack.restype = ctypes.c_int64
+    L.oracle_kv_unpack.argtypes = [_u16p, _i32p, ctypes.c_int64, _u16p, _u16p, ctypes.c_int64, ctypes.c_int64]
+    L.oracle_kv_unpack.restype = ctypes.c_int64
     L.oracle_attend_dense.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int64, ctypes.c_int32,
                                       ctypes.c_int64, ctypes.c_double, _f64p, _f64p, _f64p, _f64p]
     L.oracle_attend_dense.restype = None
@@ -132,6 +137,28 @@ def gather_kv(cache, bt_row, seq_len: int, kv_head: int = -1) -> np.ndarray:
     if rc:
         raise ValueError("block id outside the pool")
     return out
+
+
+def kv_pack(k_cache, v_cache, block_ids) -> np.ndarray:
+    """Staging [n, 2, block_elems] (bf16 bits) of whole blocks block_ids (zeros for ids outside the pool)."""
+    kc, vc = _c(k_cache, np.uint16), _c(v_cache, np.uint16)
+    NB = kc.shape[0]
+    elems = int(np.prod(kc.shape[1:]))
+    ids = _c(block_ids, np.int32)
+    out = np.zeros((len(ids), 2, elems), dtype=np.uint16)
+    _load().oracle_kv_pack(kc.reshape(-1), vc.reshape(-1), NB, elems, ids, len(ids), out.reshape(-1))
+    return out
+
+
+def kv_unpack(staging, block_ids, k_cache, v_cache):
+    """Copies of both pools with staging entry i written over block block_ids[i] (ids outside skipped)."""
+    kc, vc = np.array(k_cache, dtype=np.uint16, copy=True), np.array(v_cache, dtype=np.uint16, copy=True)
+    NB = kc.shape[0]
+    elems = int(np.prod(kc.shape[1:]))
+    ids = _c(block_ids, np.int32)
+    _load().oracle_kv_unpack(_c(staging, np.uint16).reshape(-1), ids, len(ids), kc.reshape(-1), vc.reshape(-1),
+                             NB, elems)
+    return kc, vc
 
 
 def attend_dense(q, K, V, scale: float):

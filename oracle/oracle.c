@@ -136,6 +136,56 @@ int oracle_gather_kv(const uint16_t *cache, int64_t num_blocks, int32_t num_kv_h
 }
 
 /* ------------------------------------------------------------------------
+ * Block pack / unpack for moving KV between a prefill instance and a decode
+ * instance (hn.213312.xyz section 二, item 5; shengyayun.com 关键实现细节
+ * item 4): whole blocks are copied to and from a staging buffer.
+ * A block is block_elems = num_kv_heads * block_size * head_dim contiguous
+ * bf16 values of a cache, whatever the order inside it.
+ * pack:   staging[i][0][:] = k_cache block ids[i], staging[i][1][:] = v block;
+ *         an id outside [0, num_blocks) gives a zero entry.
+ * unpack: k_cache block ids[i] = staging[i][0][:], v block = staging[i][1][:];
+ *         an id outside the pool is skipped.
+ * Both return the number of ids outside the pool.
+ * ---------------------------------------------------------------------- */
+int64_t oracle_kv_pack(const uint16_t *k_cache, const uint16_t *v_cache, int64_t num_blocks,
+                       int64_t block_elems, const int32_t *ids, int64_t n, uint16_t *staging)
+{
+    int64_t bad = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        uint16_t *dk = staging + (2 * i) * block_elems;
+        uint16_t *dv = staging + (2 * i + 1) * block_elems;
+        int64_t b = ids[i];
+        if (b < 0 || b >= num_blocks) {
+            memset(dk, 0, sizeof(uint16_t) * (size_t)block_elems);
+            memset(dv, 0, sizeof(uint16_t) * (size_t)block_elems);
+            ++bad;
+            continue;
+        }
+        memcpy(dk, k_cache + b * block_elems, sizeof(uint16_t) * (size_t)block_elems);
+        memcpy(dv, v_cache + b * block_elems, sizeof(uint16_t) * (size_t)block_elems);
+    }
+    return bad;
+}
+
+int64_t oracle_kv_unpack(const uint16_t *staging, const int32_t *ids, int64_t n, uint16_t *k_cache,
+                         uint16_t *v_cache, int64_t num_blocks, int64_t block_elems)
+{
+    int64_t bad = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t b = ids[i];
+        if (b < 0 || b >= num_blocks) {
+            ++bad;
+            continue;
+        }
+        memcpy(k_cache + b * block_elems, staging + (2 * i) * block_elems,
+               sizeof(uint16_t) * (size_t)block_elems);
+        memcpy(v_cache + b * block_elems, staging + (2 * i + 1) * block_elems,
+               sizeof(uint16_t) * (size_t)block_elems);
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------
  * Dense attention of one query row over n contiguous keys (the definition):
  *   s_j = scale * sum_d q[d] * K[j][d]
  *   w_j = exp(s_j - max_s) / sum_i exp(s_i - max_s)

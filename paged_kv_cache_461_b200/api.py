@@ -28,7 +28,10 @@ DEVICE_WAIT_TIMEOUT = 4
 # every symbol include/pa.h declares
 EXPORTED = ("pa_abi_version", "pa_status_string", "pa_kv_write", "pa_build_slot_mapping", "pa_workspace_size",
             "pa_workspace_size_ex", "pa_attention_mixed", "pa_attention_mixed_ex", "pa_attention_mixed_noalloc",
-            "pa_merge_attn_states", "pa_debug_gather_kv")
+            "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack", "pa_merge_attn_states", "pa_debug_gather_kv")
+LAYOUT_HND = 0   # cache [num_blocks, num_kv_heads, 16, head_dim]
+LAYOUT_NHD = 1   # cache [num_blocks, 16, num_kv_heads, head_dim]
+_LAYOUTS = {"HND": LAYOUT_HND, "NHD": LAYOUT_NHD}
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -40,7 +43,7 @@ class PaError(RuntimeError):
 
 class CacheDesc(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int64), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("block_size", ctypes.c_int32)]
+                ("block_size", ctypes.c_int32), ("layout", ctypes.c_int32)]
 
 
 class AttnOptions(ctypes.Structure):
@@ -74,10 +77,16 @@ def lib():
         L.pa_attention_mixed.argtypes = attn + [_vp]
         L.pa_attention_mixed_ex.argtypes = attn + [ctypes.POINTER(AttnOptions), _vp]
         L.pa_attention_mixed_noalloc.argtypes = attn[:-2] + [ctypes.POINTER(AttnOptions), _vp]
+        L.pa_attention_decode_fused.argtypes = [_vp, _i32, _vp, _vp, _i64, _vp, _vp, ctypes.POINTER(CacheDesc), _vp,
+                                                _vp, _vp, _i32, _i32, _i32, _i32, _i32, ctypes.c_float, _vp, _vp,
+                                                _vp, _sz, ctypes.POINTER(AttnOptions), _vp]
+        L.pa_kv_pack.argtypes = [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _i32, _vp, _vp]
+        L.pa_kv_unpack.argtypes = [_vp, _vp, _i32, _vp, _vp, ctypes.POINTER(CacheDesc), _vp]
         L.pa_merge_attn_states.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
         L.pa_debug_gather_kv.argtypes = [_vp, ctypes.POINTER(CacheDesc), _vp, _i32, _vp, _vp]
         for name in ("pa_kv_write", "pa_build_slot_mapping", "pa_attention_mixed", "pa_attention_mixed_ex",
-                     "pa_attention_mixed_noalloc", "pa_merge_attn_states", "pa_debug_gather_kv"):
+                     "pa_attention_mixed_noalloc", "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack",
+                     "pa_merge_attn_states", "pa_debug_gather_kv"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -98,9 +107,15 @@ def _stream(stream=None):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def cache_desc(k_cache: torch.Tensor) -> CacheDesc:
-    NB, Hkv, bs, D = k_cache.shape
-    return CacheDesc(NB, Hkv, D, bs)
+def cache_desc(k_cache: torch.Tensor, layout: str = "HND") -> CacheDesc:
+    """Descriptor of a cache tensor: HND [NB, Hkv, 16, D] or NHD [NB, 16, Hkv, D]."""
+    if layout == "HND":
+        NB, Hkv, bs, D = k_cache.shape
+    elif layout == "NHD":
+        NB, bs, Hkv, D = k_cache.shape
+    else:
+        raise ValueError(f"unknown cache layout {layout!r}")
+    return CacheDesc(NB, Hkv, D, bs, _LAYOUTS[layout])
 
 
 def _opts(kv_split_tokens: int, decode_max_query_len: int = 0) -> Optional[AttnOptions]:
@@ -124,7 +139,7 @@ def abi_version() -> int:
 
 
 def kv_write(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, k_cache: torch.Tensor,
-             v_cache: torch.Tensor, stream=None) -> None:
+             v_cache: torch.Tensor, stream=None, layout: str = "HND") -> None:
     """pa_kv_write: k_new/v_new [T, Hkv, D] (rows may be strided), slot_mapping int64 [T]."""
     _need(k_new, torch.bfloat16, "k_new")
     _need(slot_mapping, torch.int64, "slot_mapping")
@@ -132,7 +147,7 @@ def kv_write(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tenso
     row_stride = k_new.stride(0) if T else k_new.shape[-1] * k_new.shape[-2]
     if k_new.stride(0) != v_new.stride(0) or k_new.stride(-1) != 1 or k_new.stride(-2) != k_new.shape[-1]:
         raise ValueError("k_new and v_new need the same row stride and contiguous [Hkv, D] rows")
-    d = cache_desc(k_cache)
+    d = cache_desc(k_cache, layout)
     _check(lib().pa_kv_write(_ptr(k_new), _ptr(v_new), row_stride, _ptr(slot_mapping), T, _ptr(k_cache),
                              _ptr(v_cache), ctypes.byref(d), _stream(stream)), "pa_kv_write")
 
@@ -148,16 +163,17 @@ def build_slot_mapping(query_start_loc: torch.Tensor, seq_lens: torch.Tensor, bl
 
 
 def workspace_size(num_seqs: int, num_tokens: int, num_q_heads: int, k_cache_or_desc, max_seq_len: int,
-                   kv_split_tokens: int = 0, decode_max_query_len: int = 0) -> int:
-    d = k_cache_or_desc if isinstance(k_cache_or_desc, CacheDesc) else cache_desc(k_cache_or_desc)
+                   kv_split_tokens: int = 0, decode_max_query_len: int = 0, layout: str = "HND") -> int:
+    d = k_cache_or_desc if isinstance(k_cache_or_desc, CacheDesc) else cache_desc(k_cache_or_desc, layout)
     o = _opts(kv_split_tokens, decode_max_query_len)
     return int(lib().pa_workspace_size_ex(num_seqs, num_tokens, num_q_heads, ctypes.byref(d), max_seq_len,
                                           ctypes.byref(o) if o else None))
 
 
 def alloc_workspace(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens=0,
-                    decode_max_query_len=0) -> torch.Tensor:
-    n = workspace_size(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len)
+                    decode_max_query_len=0, layout: str = "HND") -> torch.Tensor:
+    n = workspace_size(num_seqs, num_tokens, num_q_heads, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len,
+                       layout)
     if n == 0:
         raise PaError(1, "pa_workspace_size")
     return torch.empty(n, dtype=torch.uint8, device=k_cache.device)
@@ -167,7 +183,8 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
                     seq_lens: torch.Tensor, block_table: torch.Tensor, max_query_len: int, max_seq_len: int,
                     softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                     lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                    kv_split_tokens: int = 0, decode_max_query_len: int = 0, stream=None) -> torch.Tensor:
+                    kv_split_tokens: int = 0, decode_max_query_len: int = 0, stream=None,
+                    layout: str = "HND") -> torch.Tensor:
     """pa_attention_mixed[_ex]: q [T, Hq, D] bf16 -> out [T, Hq, D] bf16 (lse [T, Hq] fp32 if given)."""
     _need(q, torch.bfloat16, "q")
     T, Hq, D = q.shape
@@ -177,8 +194,8 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
-        workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len)
-    d = cache_desc(k_cache)
+        workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len, layout)
+    d = cache_desc(k_cache, layout)
     o = _opts(kv_split_tokens, decode_max_query_len)
     _check(lib().pa_attention_mixed_ex(_ptr(q), Hq, _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
                                        _ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
@@ -193,7 +210,7 @@ def attention_mixed_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
                             query_start_loc: torch.Tensor, seq_lens: torch.Tensor, block_table: torch.Tensor,
                             max_query_len: int, max_seq_len: int, softmax_scale: Optional[float] = None,
                             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                            kv_split_tokens: int = 0, stream=None) -> torch.Tensor:
+                            kv_split_tokens: int = 0, stream=None, layout: str = "HND") -> torch.Tensor:
     """pa_attention_mixed_noalloc: like attention_mixed but with the library's built-in scratch
     (for callers that cannot allocate a workspace; calls that overlap on the GPU race on it)."""
     _need(q, torch.bfloat16, "q")
@@ -203,7 +220,7 @@ def attention_mixed_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
         softmax_scale = 1.0 / math.sqrt(D)
     if out is None:
         out = torch.empty_like(q)
-    d = cache_desc(k_cache)
+    d = cache_desc(k_cache, layout)
     o = _opts(kv_split_tokens)
     _check(lib().pa_attention_mixed_noalloc(_ptr(q), Hq, _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
                                             _ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
@@ -212,6 +229,63 @@ def attention_mixed_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
                                             ctypes.byref(o) if o else None, _stream(stream)),
            "pa_attention_mixed_noalloc")
     return out
+
+
+def attention_decode_fused(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
+                           v_cache: torch.Tensor, query_start_loc: torch.Tensor, seq_lens: torch.Tensor,
+                           block_table: torch.Tensor, max_query_len: int, max_seq_len: int,
+                           softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                           lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                           kv_split_tokens: int = 0, decode_max_query_len: int = 0, stream=None,
+                           layout: str = "HND") -> torch.Tensor:
+    """pa_attention_decode_fused: writes k_new/v_new [T, Hkv, D] (rows may be strided) into their
+    slots and attends, in the decode kernel; every request must be decode-shaped."""
+    _need(q, torch.bfloat16, "q")
+    _need(k_new, torch.bfloat16, "k_new")
+    T, Hq, D = q.shape
+    R = seq_lens.shape[0]
+    if k_new.stride(0) != v_new.stride(0) or k_new.stride(-1) != 1 or k_new.stride(-2) != k_new.shape[-1]:
+        raise ValueError("k_new and v_new need the same row stride and contiguous [Hkv, D] rows")
+    row_stride = k_new.stride(0) if T else k_new.shape[-1] * k_new.shape[-2]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len, layout)
+    d = cache_desc(k_cache, layout)
+    o = _opts(kv_split_tokens, decode_max_query_len)
+    _check(lib().pa_attention_decode_fused(_ptr(q), Hq, _ptr(k_new), _ptr(v_new), row_stride, _ptr(k_cache),
+                                           _ptr(v_cache), ctypes.byref(d), _ptr(query_start_loc), _ptr(seq_lens),
+                                           _ptr(block_table), block_table.stride(0), R, T, int(max_query_len),
+                                           int(max_seq_len), float(softmax_scale), _ptr(out), _ptr(lse),
+                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                           ctypes.byref(o) if o else None, _stream(stream)),
+           "pa_attention_decode_fused")
+    return out
+
+
+def kv_pack(k_cache: torch.Tensor, v_cache: torch.Tensor, block_ids: torch.Tensor,
+            staging: Optional[torch.Tensor] = None, stream=None, layout: str = "HND") -> torch.Tensor:
+    """pa_kv_pack: whole blocks block_ids (int32) -> staging bf16 [n, 2, block_elems]."""
+    _need(block_ids, torch.int32, "block_ids")
+    d = cache_desc(k_cache, layout)
+    n = block_ids.shape[0]
+    elems = d.num_kv_heads * d.block_size * d.head_dim
+    if staging is None:
+        staging = torch.empty((n, 2, elems), dtype=k_cache.dtype, device=k_cache.device)
+    _check(lib().pa_kv_pack(_ptr(k_cache), _ptr(v_cache), ctypes.byref(d), _ptr(block_ids), n, _ptr(staging),
+                            _stream(stream)), "pa_kv_pack")
+    return staging
+
+
+def kv_unpack(staging: torch.Tensor, block_ids: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              stream=None, layout: str = "HND") -> None:
+    """pa_kv_unpack: staging bf16 [n, 2, block_elems] -> whole blocks block_ids of the caches."""
+    _need(block_ids, torch.int32, "block_ids")
+    d = cache_desc(k_cache, layout)
+    _check(lib().pa_kv_unpack(_ptr(staging), _ptr(block_ids), block_ids.shape[0], _ptr(k_cache), _ptr(v_cache),
+                              ctypes.byref(d), _stream(stream)), "pa_kv_unpack")
 
 
 def merge_attn_states(part_out: torch.Tensor, part_lse: torch.Tensor, parts_per_row: Optional[torch.Tensor] = None,
@@ -226,10 +300,10 @@ def merge_attn_states(part_out: torch.Tensor, part_lse: torch.Tensor, parts_per_
     return out
 
 
-def debug_gather_kv(cache: torch.Tensor, bt_row: torch.Tensor, seq_len: int, stream=None) -> torch.Tensor:
-    NB, Hkv, bs, D = cache.shape
-    out = torch.empty((seq_len, Hkv, D), dtype=cache.dtype, device=cache.device)
-    d = cache_desc(cache)
+def debug_gather_kv(cache: torch.Tensor, bt_row: torch.Tensor, seq_len: int, stream=None,
+                    layout: str = "HND") -> torch.Tensor:
+    d = cache_desc(cache, layout)
+    out = torch.empty((seq_len, d.num_kv_heads, d.head_dim), dtype=cache.dtype, device=cache.device)
     _check(lib().pa_debug_gather_kv(_ptr(cache), ctypes.byref(d), _ptr(bt_row), seq_len, _ptr(out),
                                     _stream(stream)), "pa_debug_gather_kv")
     return out

@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpa_b200.so")
 SOURCES = ["pa_api.cu", "kv_write.cu", "plan_merge.cu", "decode.cu", "prefill.cu", "pa_noalloc.cu"]
-HEADERS = ["ptx.cuh", "pa_internal.cuh"]
+HEADERS = ["ptx.cuh", "tcgen05.cuh", "pa_internal.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

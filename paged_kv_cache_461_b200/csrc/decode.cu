@@ -112,17 +112,27 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
         if (lane == 0) {
             const int stage = k % kDecStages;
             const uint32_t bar = wbar + stage * 8;
+            // HND: 2-D map {D, blocks*Hkv*16}, row (bid*Hkv + h)*16;  NHD: 3-D map {D, Hkv, blocks*16},
+            // (head h, token row bid*16).  Either way the box is 16 rows x 64 columns.
             int y = -kBlockSize; // fully out of bounds: TMA fills zeros
             if ((unsigned)bid < (unsigned long long)p.num_blocks)
-                y = (bid * p.Hkv + h) * kBlockSize;
+                y = (p.nhd ? bid : bid * p.Hkv + h) * kBlockSize;
             else
                 atomicOr(&p.hdr->status, PA_DEVICE_BAD_BLOCK);
             mbar_arrive_expect_tx(bar, Cfg::kStage);
             const uint32_t sk = wbase_s + stage * Cfg::kStage;
+            if (p.nhd) {
 #pragma unroll
-            for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-                tma_load_2d(sk + hf * Cfg::kBox, &tm_k, hf * 64, y, bar);
-                tma_load_2d(sk + Cfg::kTile + hf * Cfg::kBox, &tm_v, hf * 64, y, bar);
+                for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+                    tma_load_3d(sk + hf * Cfg::kBox, &tm_k, hf * 64, h, y, bar);
+                    tma_load_3d(sk + Cfg::kTile + hf * Cfg::kBox, &tm_v, hf * 64, h, y, bar);
+                }
+            } else {
+#pragma unroll
+                for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+                    tma_load_2d(sk + hf * Cfg::kBox, &tm_k, hf * 64, y, bar);
+                    tma_load_2d(sk + Cfg::kTile + hf * Cfg::kBox, &tm_v, hf * 64, y, bar);
+                }
             }
         }
     };
@@ -186,6 +196,32 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
         const int j0 = k_begin + (warp + kDecWarps * k) * kBlockSize;
         const uint32_t sK = wbase_s + stage * Cfg::kStage;
         const uint32_t sV = sK + Cfg::kTile;
+        if (p.k_new != nullptr) {
+            // fused KV write: this block's rows at positions ctx..L-1 are the step's new tokens.
+            // Store them into the cache and over the (stale) rows the TMA just brought in.
+            const int lo = max(j0, ctx), hi = min(j0 + kBlockSize, L);
+            if (lo < hi) {
+                const int64_t bidw = bt_row[j0 / kBlockSize];
+                if (bidw >= 0 && bidw < p.num_blocks) {
+                    constexpr int kCh = D / 8; // 16-byte chunks per row
+                    uint8_t *tile = wbase + stage * Cfg::kStage;
+                    for (int i = lane; i < (hi - lo) * 2 * kCh; i += 32) {
+                        const int c = i % kCh, kv = (i / kCh) & 1, pos = lo + i / (2 * kCh);
+                        const int64_t t = qs + (pos - ctx);
+                        const int row = pos - j0;
+                        const uint4 val = *reinterpret_cast<const uint4 *>((kv ? p.v_new : p.k_new) +
+                                                                            t * p.new_row_stride + h * D + c * 8);
+                        *reinterpret_cast<uint4 *>(tile + kv * Cfg::kTile + tile_off(row, c)) = val;
+                        const int64_t e = p.nhd ? ((bidw * kBlockSize + row) * p.Hkv + h) * D + c * 8
+                                                : ((bidw * p.Hkv + h) * kBlockSize + row) * D + c * 8;
+                        *reinterpret_cast<uint4 *>((kv ? p.v_cache_w : p.k_cache_w) + e) = val;
+                    }
+                    // the stage is refilled by TMA (async proxy) after these generic writes
+                    fence_proxy_async_smem();
+                }
+            }
+            __syncwarp();
+        }
 
         // ---- S^T[16 keys x 8NT cols] = K . Q^T
         float s[NT][4];

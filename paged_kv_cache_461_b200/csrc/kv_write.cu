@@ -1,8 +1,13 @@
 // kv_write.cu -- the KV-cache write (scatter of this step's K/V rows into their
-// 16-token blocks through the slot mapping), the slot-mapping builder and the
-// debug gather.  All three are pure data movement, bound by HBM bandwidth:
-// each warp moves whole (token, head) rows with 16-byte vector accesses, so
-// every load and store is a full 32-byte sector run.
+// 16-token blocks through the slot mapping), the slot-mapping builder, the
+// debug gather and the whole-block pack / unpack to a staging buffer.  All are
+// pure data movement, bound by HBM bandwidth: each warp moves whole (token,
+// head) rows with 16-byte vector accesses, so every load and store is a full
+// 32-byte sector run.
+//
+// Inside a block the element (token o, kv head h, dim d) sits at
+// h*head_stride + o*tok_stride + d: HND (head-major) has head_stride = 16*D,
+// tok_stride = D; NHD (token-major) has head_stride = D, tok_stride = Hkv*D.
 //
 // Semantics follow the model-runner step restated on hn.213312.xyz (section 一,
 // "前向传播"): prepare-inputs builds positions and the slot mapping, then the
@@ -20,7 +25,8 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const uint16_t *__restric
                                                        const uint16_t *__restrict__ v_new, int64_t row_stride,
                                                        const int64_t *__restrict__ slots, int num_tokens,
                                                        uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
-                                                       int64_t num_blocks, int Hkv, int D)
+                                                       int64_t num_blocks, int Hkv, int D, int head_stride,
+                                                       int tok_stride)
 {
     using Vec = typename std::conditional<VEC == 8, uint4, uint16_t>::type;
     const int lane = threadIdx.x & 31;
@@ -40,7 +46,7 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const uint16_t *__restric
         for (int i = lane; i < vec_per_tok; i += 32) {
             const int h = i / vec_per_row;
             const int e = (i - h * vec_per_row) * VEC;
-            const int64_t dst = ((blk * Hkv + h) * kBlockSize + off) * (int64_t)D + e;
+            const int64_t dst = blk * ((int64_t)Hkv * kBlockSize * D) + h * head_stride + off * tok_stride + e;
             const Vec kv = *reinterpret_cast<const Vec *>(ks + (int64_t)h * D + e);
             const Vec vv = *reinterpret_cast<const Vec *>(vs + (int64_t)h * D + e);
             *reinterpret_cast<Vec *>(k_cache + dst) = kv;
@@ -72,7 +78,8 @@ __global__ void slot_mapping_kernel(const int32_t *__restrict__ qsl, const int32
 
 // One warp per token of the request: copy its Hkv rows into out[j].
 __global__ void gather_kernel(const uint16_t *__restrict__ cache, int64_t num_blocks, int Hkv, int D,
-                              const int32_t *__restrict__ bt_row, int seq_len, uint16_t *__restrict__ out)
+                              int head_stride, int tok_stride, const int32_t *__restrict__ bt_row, int seq_len,
+                              uint16_t *__restrict__ out)
 {
     const int lane = threadIdx.x & 31;
     const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -86,17 +93,83 @@ __global__ void gather_kernel(const uint16_t *__restrict__ cache, int64_t num_bl
         const int h = i / D, d = i - h * D;
         uint16_t v = 0;
         if (ok)
-            v = cache[((blk * Hkv + h) * kBlockSize + off) * (int64_t)D + d];
+            v = cache[blk * ((int64_t)Hkv * kBlockSize * D) + h * head_stride + off * tok_stride + d];
         out[(int64_t)j * n + i] = v;
+    }
+}
+
+// Whole-block copies between the caches and a staging buffer [num_ids][2][bv] of 16-byte
+// vectors (bv vectors per block).  One unit = (entry i, cache kv) = staging row 2i+kv; CTAs
+// stride over units and each CTA's threads over the unit's vectors, four in flight per
+// thread.  PACK: cache -> staging (an id outside the pool gives zeros); otherwise
+// staging -> cache (an id outside the pool is skipped).
+template <bool PACK>
+__global__ void __launch_bounds__(256) kv_block_copy_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                                                            int64_t num_blocks, int bv,
+                                                            const int32_t *__restrict__ ids, int64_t n_units,
+                                                            uint4 *__restrict__ staging)
+{
+    constexpr int kU = 4;
+    for (int64_t unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+        const int64_t bid = ids[unit >> 1];
+        const bool ok = bid >= 0 && bid < num_blocks;
+        if (!PACK && !ok)
+            continue;
+        uint4 *cache = ((unit & 1) ? v_cache : k_cache) + (ok ? bid : 0) * (int64_t)bv;
+        uint4 *stg = staging + unit * (int64_t)bv;
+        for (int base = threadIdx.x; base < bv; base += blockDim.x * kU) {
+            uint4 val[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int v = base + u * (int)blockDim.x;
+                val[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (v < bv && (!PACK || ok))
+                    val[u] = PACK ? cache[v] : stg[v];
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int v = base + u * (int)blockDim.x;
+                if (v < bv) {
+                    if (PACK)
+                        stg[v] = val[u];
+                    else
+                        cache[v] = val[u];
+                }
+            }
+        }
     }
 }
 
 } // namespace
 
+cudaError_t launch_kv_pack(const void *k_cache, const void *v_cache, int64_t num_blocks, int64_t block_elems,
+                           const int32_t *ids, int num_ids, void *staging, int num_sms, cudaStream_t s)
+{
+    const int64_t units = 2 * (int64_t)num_ids;
+    const unsigned grid = (unsigned)(units < (int64_t)num_sms * 8 ? units : (int64_t)num_sms * 8);
+    kv_block_copy_kernel<true><<<grid, 256, 0, s>>>(
+        const_cast<uint4 *>(static_cast<const uint4 *>(k_cache)), const_cast<uint4 *>(static_cast<const uint4 *>(v_cache)),
+        num_blocks, (int)(block_elems / 8), ids, units, static_cast<uint4 *>(staging));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kv_unpack(const void *staging, const int32_t *ids, int num_ids, void *k_cache, void *v_cache,
+                             int64_t num_blocks, int64_t block_elems, int num_sms, cudaStream_t s)
+{
+    const int64_t units = 2 * (int64_t)num_ids;
+    const unsigned grid = (unsigned)(units < (int64_t)num_sms * 8 ? units : (int64_t)num_sms * 8);
+    kv_block_copy_kernel<false><<<grid, 256, 0, s>>>(static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache),
+                                                     num_blocks, (int)(block_elems / 8), ids, units,
+                                                     const_cast<uint4 *>(static_cast<const uint4 *>(staging)));
+    return cudaGetLastError();
+}
+
 cudaError_t launch_kv_write(const void *k_new, const void *v_new, int64_t row_stride, const int64_t *slots,
                             int num_tokens, void *k_cache, void *v_cache, int64_t num_blocks, int Hkv, int D,
-                            cudaStream_t s)
+                            int nhd, cudaStream_t s)
 {
+    const int head_stride = nhd ? D : kBlockSize * D;
+    const int tok_stride = nhd ? Hkv * D : D;
     const bool vec_ok = ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new) |
                           reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) % 16 == 0) &&
                         (row_stride % 8 == 0) && (D % 8 == 0);
@@ -110,11 +183,13 @@ cudaError_t launch_kv_write(const void *k_new, const void *v_new, int64_t row_st
     if (vec_ok)
         kv_write_kernel<8><<<(unsigned)blocks, threads, 0, s>>>(
             static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new), row_stride, slots, num_tokens,
-            static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache), num_blocks, Hkv, D);
+            static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache), num_blocks, Hkv, D, head_stride,
+            tok_stride);
     else
         kv_write_kernel<1><<<(unsigned)blocks, threads, 0, s>>>(
             static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new), row_stride, slots, num_tokens,
-            static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache), num_blocks, Hkv, D);
+            static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache), num_blocks, Hkv, D, head_stride,
+            tok_stride);
     return cudaGetLastError();
 }
 
@@ -125,13 +200,14 @@ cudaError_t launch_slot_mapping(const int32_t *qsl, const int32_t *seq_lens, con
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D, const int32_t *bt_row, int seq_len,
-                          void *out, cudaStream_t s)
+cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D, int nhd, const int32_t *bt_row,
+                          int seq_len, void *out, cudaStream_t s)
 {
     const int threads = 256;
     const int blocks = (seq_len + 7) / 8;
-    gather_kernel<<<blocks, threads, 0, s>>>(static_cast<const uint16_t *>(cache), num_blocks, Hkv, D, bt_row,
-                                             seq_len, static_cast<uint16_t *>(out));
+    gather_kernel<<<blocks, threads, 0, s>>>(static_cast<const uint16_t *>(cache), num_blocks, Hkv, D,
+                                             nhd ? D : kBlockSize * D, nhd ? Hkv * D : D, bt_row, seq_len,
+                                             static_cast<uint16_t *>(out));
     return cudaGetLastError();
 }
 

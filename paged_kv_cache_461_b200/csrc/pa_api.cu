@@ -23,6 +23,10 @@ bool cache_desc_ok(const pa_cache_desc_t *c, pa_status_t *why)
         *why = PA_ERR_INVALID_ARG;
         return false;
     }
+    if (c->layout != PA_LAYOUT_HND && c->layout != PA_LAYOUT_NHD) {
+        *why = PA_ERR_INVALID_ARG;
+        return false;
+    }
     if (c->block_size != kBlockSize || (c->head_dim != 64 && c->head_dim != 128)) {
         *why = PA_ERR_UNSUPPORTED;
         return false;
@@ -194,7 +198,7 @@ pa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ER
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 1; }
+int32_t pa_abi_version(void) { return 2; }
 
 const char *pa_status_string(pa_status_t s)
 {
@@ -228,7 +232,7 @@ pa_status_t pa_kv_write(const void *k_new, const void *v_new, int64_t new_row_st
         return PA_ERR_INVALID_ARG;
     return cuda_status(launch_kv_write(k_new, v_new, new_row_stride, slot_mapping, num_tokens, k_cache, v_cache,
                                        cache->num_blocks, cache->num_kv_heads, cache->head_dim,
-                                       reinterpret_cast<cudaStream_t>(stream)));
+                                       cache->layout == PA_LAYOUT_NHD, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 pa_status_t pa_build_slot_mapping(const int32_t *query_start_loc, const int32_t *seq_lens, const int32_t *block_table,
@@ -261,12 +265,22 @@ size_t pa_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t num_q_hea
     return pa_workspace_size_ex(num_seqs, num_tokens, num_q_heads, cache, max_seq_len, nullptr);
 }
 
-pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, const void *k_cache, const void *v_cache,
-                                  const pa_cache_desc_t *cache, const int32_t *query_start_loc,
-                                  const int32_t *seq_lens, const int32_t *block_table, int32_t bt_stride,
-                                  int32_t num_seqs, int32_t num_tokens, int32_t max_query_len, int32_t max_seq_len,
-                                  float softmax_scale, void *out, float *lse, void *workspace,
-                                  size_t workspace_bytes, const pa_attn_options_t *options, pa_stream_t stream)
+} // extern "C"
+
+namespace {
+
+// New K/V rows the decode kernel stores itself (pa_attention_decode_fused).
+struct FusedWrite {
+    const void *k_new, *v_new;
+    int64_t row_stride;
+};
+
+pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cache, const void *v_cache,
+                           const pa_cache_desc_t *cache, const int32_t *query_start_loc, const int32_t *seq_lens,
+                           const int32_t *block_table, int32_t bt_stride, int32_t num_seqs, int32_t num_tokens,
+                           int32_t max_query_len, int32_t max_seq_len, float softmax_scale, void *out, float *lse,
+                           void *workspace, size_t workspace_bytes, const pa_attn_options_t *options,
+                           const FusedWrite *fw, pa_stream_t stream)
 {
     Plan P;
     pa_status_t why;
@@ -292,9 +306,25 @@ pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, const void
         return PA_ERR_WORKSPACE_TOO_SMALL;
 
     const int Hkv = cache->num_kv_heads;
+    const bool nhd = cache->layout == PA_LAYOUT_NHD;
+    if (fw) {
+        // every request must be decode-shaped: the prefill kernel reads the new rows from the cache
+        if ((int64_t)max_query_len * P.G > P.dec_rows_cap || P.NT == 0)
+            return PA_ERR_UNSUPPORTED;
+        if (!fw->k_new || !fw->v_new || fw->row_stride < (int64_t)Hkv * D)
+            return PA_ERR_INVALID_ARG;
+        if (!aligned16(fw->k_new) || !aligned16(fw->v_new) || fw->row_stride % 8 != 0)
+            return PA_ERR_UNSUPPORTED;
+    }
+    // HND: 2-D {D, blocks*Hkv*16} with 16-row boxes;  NHD: 3-D {D, Hkv, blocks*16} with {64, 1, 16} boxes
     const uint64_t kv_rows = (uint64_t)cache->num_blocks * Hkv * kBlockSize;
+    const uint64_t tok_rows = (uint64_t)cache->num_blocks * kBlockSize;
     CUtensorMap tk, tv;
-    if (!get_map(k_cache, 2, D, kv_rows, 1, kBlockSize, 1, &tk) || !get_map(v_cache, 2, D, kv_rows, 1, kBlockSize, 1, &tv))
+    const bool maps_ok =
+        nhd ? get_map(k_cache, 3, D, (uint64_t)Hkv, tok_rows, 1, kBlockSize, &tk) &&
+                  get_map(v_cache, 3, D, (uint64_t)Hkv, tok_rows, 1, kBlockSize, &tv)
+            : get_map(k_cache, 2, D, kv_rows, 1, kBlockSize, 1, &tk) && get_map(v_cache, 2, D, kv_rows, 1, kBlockSize, 1, &tv);
+    if (!maps_ok)
         return PA_ERR_CUDA;
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -326,6 +356,14 @@ pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, const void
     p.max_splits = P.max_splits;
     p.QD = P.QD;
     p.dec_rows_cap = P.dec_rows_cap;
+    p.nhd = nhd;
+    if (fw) {
+        p.k_new = static_cast<const uint16_t *>(fw->k_new);
+        p.v_new = static_cast<const uint16_t *>(fw->v_new);
+        p.new_row_stride = fw->row_stride;
+        p.k_cache_w = static_cast<uint16_t *>(const_cast<void *>(k_cache));
+        p.v_cache_w = static_cast<uint16_t *>(const_cast<void *>(v_cache));
+    }
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = launch_plan(p, s);
@@ -351,6 +389,85 @@ pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, const void
             return PA_ERR_CUDA;
     }
     return PA_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, const void *k_cache, const void *v_cache,
+                                  const pa_cache_desc_t *cache, const int32_t *query_start_loc,
+                                  const int32_t *seq_lens, const int32_t *block_table, int32_t bt_stride,
+                                  int32_t num_seqs, int32_t num_tokens, int32_t max_query_len, int32_t max_seq_len,
+                                  float softmax_scale, void *out, float *lse, void *workspace,
+                                  size_t workspace_bytes, const pa_attn_options_t *options, pa_stream_t stream)
+{
+    return attention_impl(q, num_q_heads, k_cache, v_cache, cache, query_start_loc, seq_lens, block_table, bt_stride,
+                          num_seqs, num_tokens, max_query_len, max_seq_len, softmax_scale, out, lse, workspace,
+                          workspace_bytes, options, nullptr, stream);
+}
+
+pa_status_t pa_attention_decode_fused(const void *q, int32_t num_q_heads, const void *k_new, const void *v_new,
+                                      int64_t new_row_stride, void *k_cache, void *v_cache,
+                                      const pa_cache_desc_t *cache, const int32_t *query_start_loc,
+                                      const int32_t *seq_lens, const int32_t *block_table, int32_t bt_stride,
+                                      int32_t num_seqs, int32_t num_tokens, int32_t max_query_len,
+                                      int32_t max_seq_len, float softmax_scale, void *out, float *lse,
+                                      void *workspace, size_t workspace_bytes, const pa_attn_options_t *options,
+                                      pa_stream_t stream)
+{
+    const FusedWrite fw{k_new, v_new, new_row_stride};
+    return attention_impl(q, num_q_heads, k_cache, v_cache, cache, query_start_loc, seq_lens, block_table, bt_stride,
+                          num_seqs, num_tokens, max_query_len, max_seq_len, softmax_scale, out, lse, workspace,
+                          workspace_bytes, options, &fw, stream);
+}
+
+pa_status_t pa_kv_pack(const void *k_cache, const void *v_cache, const pa_cache_desc_t *cache,
+                       const int32_t *block_ids, int32_t num_ids, void *staging, pa_stream_t stream)
+{
+    pa_status_t why;
+    if (!cache_desc_ok(cache, &why))
+        return why;
+    if (num_ids < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_ids == 0)
+        return PA_OK;
+    if (!k_cache || !v_cache || !block_ids || !staging)
+        return PA_ERR_INVALID_ARG;
+    const int64_t block_elems = (int64_t)cache->num_kv_heads * kBlockSize * cache->head_dim;
+    const size_t cache_bytes = (size_t)cache->num_blocks * block_elems * 2;
+    const size_t stage_bytes = (size_t)num_ids * 2 * block_elems * 2;
+    if (ranges_overlap(staging, stage_bytes, k_cache, cache_bytes) ||
+        ranges_overlap(staging, stage_bytes, v_cache, cache_bytes))
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(staging) || !aligned16(block_ids))
+        return PA_ERR_UNSUPPORTED;
+    return cuda_status(launch_kv_pack(k_cache, v_cache, cache->num_blocks, block_elems, block_ids, num_ids, staging,
+                                      device_sms(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+pa_status_t pa_kv_unpack(const void *staging, const int32_t *block_ids, int32_t num_ids, void *k_cache,
+                         void *v_cache, const pa_cache_desc_t *cache, pa_stream_t stream)
+{
+    pa_status_t why;
+    if (!cache_desc_ok(cache, &why))
+        return why;
+    if (num_ids < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_ids == 0)
+        return PA_OK;
+    if (!k_cache || !v_cache || !block_ids || !staging)
+        return PA_ERR_INVALID_ARG;
+    const int64_t block_elems = (int64_t)cache->num_kv_heads * kBlockSize * cache->head_dim;
+    const size_t cache_bytes = (size_t)cache->num_blocks * block_elems * 2;
+    const size_t stage_bytes = (size_t)num_ids * 2 * block_elems * 2;
+    if (ranges_overlap(staging, stage_bytes, k_cache, cache_bytes) ||
+        ranges_overlap(staging, stage_bytes, v_cache, cache_bytes))
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(staging) || !aligned16(block_ids))
+        return PA_ERR_UNSUPPORTED;
+    return cuda_status(launch_kv_unpack(staging, block_ids, num_ids, k_cache, v_cache, cache->num_blocks, block_elems,
+                                        device_sms(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 pa_status_t pa_attention_mixed(const void *q, int32_t num_q_heads, const void *k_cache, const void *v_cache,
@@ -394,8 +511,9 @@ pa_status_t pa_debug_gather_kv(const void *cache_ptr, const pa_cache_desc_t *cac
         return PA_OK;
     if (!cache_ptr || !bt_row || !out)
         return PA_ERR_INVALID_ARG;
-    return cuda_status(launch_gather(cache_ptr, cache->num_blocks, cache->num_kv_heads, cache->head_dim, bt_row,
-                                     seq_len, out, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_gather(cache_ptr, cache->num_blocks, cache->num_kv_heads, cache->head_dim,
+                                     cache->layout == PA_LAYOUT_NHD, bt_row, seq_len, out,
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 } // extern "C"

@@ -64,16 +64,25 @@ struct AttnParams {
     float *part_o;              // [num_seqs*QD*Hq*max_splits, D]
     float *part_lse;            // [num_seqs*QD*Hq*max_splits]
     int split_tokens, max_splits, QD, dec_rows_cap;
+    int nhd;                    // cache layout PA_LAYOUT_NHD (else HND)
+    // fused KV write (pa_attention_decode_fused); k_new == nullptr otherwise
+    const uint16_t *k_new, *v_new;
+    int64_t new_row_stride;     // elements
+    uint16_t *k_cache_w, *v_cache_w;
 };
 
 // launchers (return cudaGetLastError() of the launch)
 cudaError_t launch_kv_write(const void *k_new, const void *v_new, int64_t row_stride, const int64_t *slots,
                             int num_tokens, void *k_cache, void *v_cache, int64_t num_blocks, int Hkv, int D,
-                            cudaStream_t s);
+                            int nhd, cudaStream_t s);
+cudaError_t launch_kv_pack(const void *k_cache, const void *v_cache, int64_t num_blocks, int64_t block_elems,
+                           const int32_t *ids, int num_ids, void *staging, int num_sms, cudaStream_t s);
+cudaError_t launch_kv_unpack(const void *staging, const int32_t *ids, int num_ids, void *k_cache, void *v_cache,
+                             int64_t num_blocks, int64_t block_elems, int num_sms, cudaStream_t s);
 cudaError_t launch_slot_mapping(const int32_t *qsl, const int32_t *seq_lens, const int32_t *bt, int bt_stride,
                                 int num_seqs, int num_tokens, int64_t *slots, cudaStream_t s);
-cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D, const int32_t *bt_row, int seq_len,
-                          void *out, cudaStream_t s);
+cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D, int nhd, const int32_t *bt_row,
+                          int seq_len, void *out, cudaStream_t s);
 cudaError_t launch_plan(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_decode(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int NT,
                           int64_t grid_units, int num_sms, cudaStream_t s);

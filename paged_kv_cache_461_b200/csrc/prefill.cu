@@ -51,8 +51,8 @@
 // never enters O.
 #include <math_constants.h>
 
-#include "ptx.cuh"
 #include "pa_internal.cuh"
+#include "tcgen05.cuh"
 
 namespace pa {
 namespace {
@@ -252,11 +252,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             for (int j = 0; j < g.n_steps; ++j, ++gs) {
                 const int st = gs & 1;
                 const int nblk = blocks_in_step(g.n_keys_all, j);
+                // HND: 2-D map, row (bid*Hkv + h)*16;  NHD: 3-D map, (head h, token row bid*16)
                 int y = -kBlockSize; // out-of-bounds box: TMA fills zeros
                 if (lane < nblk) {
                     const int bid = bt_row[j * kStepBlocks + lane];
                     if ((unsigned)bid < (unsigned long long)p.num_blocks)
-                        y = (bid * p.Hkv + g.h) * kBlockSize;
+                        y = (p.nhd ? bid : bid * p.Hkv + g.h) * kBlockSize;
                     else
                         atomicOr(&p.hdr->status, PA_DEVICE_BAD_BLOCK);
                 }
@@ -272,9 +273,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 __syncwarp();
                 if (lane < nblk)
 #pragma unroll
-                    for (int hf = 0; hf < Cfg::kHalves; ++hf)
-                        tma_load_2d(sK0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128),
-                                    &tm_k, hf * 64, y, bar + (B_KF + st) * 8);
+                    for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+                        const uint32_t dst = sK0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128);
+                        if (p.nhd)
+                            tma_load_3d(dst, &tm_k, hf * 64, g.h, y, bar + (B_KF + st) * 8);
+                        else
+                            tma_load_2d(dst, &tm_k, hf * 64, y, bar + (B_KF + st) * 8);
+                    }
                 // V into stage st once the V two steps back is consumed
                 if (gs >= 2 && !mbar_wait_warp(bar + (B_VE + st) * 8, ph_prev, abort_flag)) {
                     ok = false;
@@ -285,9 +290,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 __syncwarp();
                 if (lane < nblk)
 #pragma unroll
-                    for (int hf = 0; hf < Cfg::kHalves; ++hf)
-                        tma_load_2d(sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128),
-                                    &tm_v, hf * 64, y, bar + (B_VF + st) * 8);
+                    for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+                        const uint32_t dst = sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128);
+                        if (p.nhd)
+                            tma_load_3d(dst, &tm_v, hf * 64, g.h, y, bar + (B_VF + st) * 8);
+                        else
+                            tma_load_2d(dst, &tm_v, hf * 64, y, bar + (B_VF + st) * 8);
+                    }
                 if (g.tail_fix && j == g.n_steps - 1) {
                     // zero the V rows past the end of the sequence in its last block
                     if (!mbar_wait_warp(bar + (B_VF + st) * 8, (gs >> 1) & 1, abort_flag)) {

@@ -43,11 +43,22 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
-class DevStep:
-    """Device copies of one step (metadata + values)."""
+def to_nhd(cache: torch.Tensor) -> torch.Tensor:
+    """[NB, Hkv, 16, D] (HND) -> contiguous [NB, 16, Hkv, D] (NHD): the same values, token-major blocks."""
+    return cache.transpose(1, 2).contiguous()
 
-    def __init__(self, layout: W.StepLayout, vals: W.StepValues, dev="cuda"):
+
+def to_hnd(cache: torch.Tensor) -> torch.Tensor:
+    return cache.transpose(1, 2).contiguous()
+
+
+class DevStep:
+    """Device copies of one step (metadata + values).  kv_layout "NHD" stores the caches
+    token-major ([NB, 16, Hkv, D]); the host values are always HND."""
+
+    def __init__(self, layout: W.StepLayout, vals: W.StepValues, dev="cuda", kv_layout="HND"):
         self.layout = layout
+        self.kv_layout = kv_layout
         self.qsl = torch.from_numpy(layout.query_start_loc).to(dev)
         self.seq_lens = torch.from_numpy(layout.seq_lens).to(dev)
         self.bt = torch.from_numpy(layout.block_table).to(dev)
@@ -58,22 +69,47 @@ class DevStep:
         else:
             self.q, self.k_new, self.v_new = vals.q, vals.k_new, vals.v_new
             self.k_cache, self.v_cache = vals.k_cache, vals.v_cache
+        if kv_layout == "NHD":
+            self.k_cache, self.v_cache = to_nhd(self.k_cache), to_nhd(self.v_cache)
 
     def write(self):
-        api.kv_write(self.k_new, self.v_new, self.slots, self.k_cache, self.v_cache)
+        api.kv_write(self.k_new, self.v_new, self.slots, self.k_cache, self.v_cache, layout=self.kv_layout)
 
-    def attend(self, kv_split_tokens=0, with_lse=True, scale=None, workspace=None, decode_max_query_len=0):
+    def _ws(self, workspace, kv_split_tokens, decode_max_query_len):
+        lay = self.layout
+        if workspace is None:
+            workspace = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, self.k_cache,
+                                            lay.max_seq_len, kv_split_tokens, decode_max_query_len,
+                                            layout=self.kv_layout)
+        return workspace
+
+    def _outs(self, with_lse):
         lay = self.layout
         lse = torch.full((lay.num_tokens, lay.num_q_heads), float("nan"), dtype=torch.float32,
                          device=self.q.device) if with_lse else None
-        out = torch.full_like(self.q, float("nan"))
-        if workspace is None:
-            workspace = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, self.k_cache,
-                                            lay.max_seq_len, kv_split_tokens, decode_max_query_len)
+        return torch.full_like(self.q, float("nan")), lse
+
+    def attend(self, kv_split_tokens=0, with_lse=True, scale=None, workspace=None, decode_max_query_len=0):
+        lay = self.layout
+        out, lse = self._outs(with_lse)
+        workspace = self._ws(workspace, kv_split_tokens, decode_max_query_len)
         api.attention_mixed(self.q, self.k_cache, self.v_cache, self.qsl, self.seq_lens, self.bt,
                             lay.max_query_len, lay.max_seq_len, softmax_scale=scale, out=out, lse=lse,
                             workspace=workspace, kv_split_tokens=kv_split_tokens,
-                            decode_max_query_len=decode_max_query_len)
+                            decode_max_query_len=decode_max_query_len, layout=self.kv_layout)
+        self.workspace = workspace
+        return out, lse
+
+    def write_and_attend_fused(self, kv_split_tokens=0, with_lse=True, scale=None, workspace=None,
+                               decode_max_query_len=0):
+        """pa_attention_decode_fused: this step's K/V written by the decode kernel itself."""
+        lay = self.layout
+        out, lse = self._outs(with_lse)
+        workspace = self._ws(workspace, kv_split_tokens, decode_max_query_len)
+        api.attention_decode_fused(self.q, self.k_new, self.v_new, self.k_cache, self.v_cache, self.qsl,
+                                   self.seq_lens, self.bt, lay.max_query_len, lay.max_seq_len, softmax_scale=scale,
+                                   out=out, lse=lse, workspace=workspace, kv_split_tokens=kv_split_tokens,
+                                   decode_max_query_len=decode_max_query_len, layout=self.kv_layout)
         self.workspace = workspace
         return out, lse
 

@@ -47,7 +47,7 @@ def test_library_exports_nothing_else(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.pa_abi_version() == 1
+    assert L.pa_abi_version() == 2
     for code, name in api.STATUS_NAMES.items():
         assert L.pa_status_string(code).decode() == name
 
@@ -147,3 +147,54 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         api.lib()
+
+
+def test_cache_layout_field(L):
+    d = _desc()
+    assert ctypes.sizeof(api.CacheDesc) == 24          # the layout field sits in what was padding
+    bad = api.CacheDesc(64, 8, 128, 16, 2)
+    assert L.pa_workspace_size(4, 4, 32, ctypes.byref(bad), 1000) == 0
+    assert L.pa_kv_write(FAKE, FAKE, 1024, FAKE, 4, FAKE, FAKE, ctypes.byref(bad), None) == 1
+    nhd = api.CacheDesc(64, 8, 128, 16, api.LAYOUT_NHD)
+    assert L.pa_workspace_size(4, 4, 32, ctypes.byref(nhd), 1000) == L.pa_workspace_size(4, 4, 32, ctypes.byref(d), 1000)
+
+
+def test_pack_unpack_host_validation(L):
+    d = _desc()
+    big = 1 << 34                                       # far from the (fake) caches
+    assert L.pa_kv_pack(FAKE, FAKE + (1 << 30), ctypes.byref(d), FAKE, 0, FAKE + big, None) == 0
+    assert L.pa_kv_pack(FAKE, FAKE + (1 << 30), ctypes.byref(d), FAKE, -1, FAKE + big, None) == 1
+    assert L.pa_kv_pack(None, FAKE + (1 << 30), ctypes.byref(d), FAKE, 3, FAKE + big, None) == 1
+    assert L.pa_kv_pack(FAKE, FAKE + (1 << 30), ctypes.byref(d), None, 3, FAKE + big, None) == 1
+    assert L.pa_kv_pack(FAKE, FAKE + (1 << 30), ctypes.byref(d), FAKE, 3, FAKE + 64, None) == 1   # staging in k_cache
+    assert L.pa_kv_pack(FAKE, FAKE + (1 << 30), ctypes.byref(d), FAKE, 3, FAKE + big + 8, None) == 2
+    assert L.pa_kv_pack(FAKE, FAKE + (1 << 30), ctypes.byref(_desc(d=96)), FAKE, 3, FAKE + big, None) == 2
+    assert L.pa_kv_unpack(FAKE + big, FAKE, -1, FAKE, FAKE + (1 << 30), ctypes.byref(d), None) == 1
+    assert L.pa_kv_unpack(FAKE + big, FAKE, 0, FAKE, FAKE + (1 << 30), ctypes.byref(d), None) == 0
+    assert L.pa_kv_unpack(FAKE + (1 << 30) + 32, FAKE, 2, FAKE, FAKE + (1 << 30), ctypes.byref(d), None) == 1
+    assert L.pa_kv_unpack(FAKE + big, FAKE, 2, FAKE + 2, FAKE + (1 << 30), ctypes.byref(d), None) == 2
+
+
+def _fused(L, **kw):
+    a = dict(q=FAKE, hq=32, kn=FAKE + (1 << 33), vn=FAKE + (1 << 33) + (1 << 28), stride=1024, k=FAKE + (1 << 31),
+             v=FAKE + (1 << 31) + (1 << 29), desc=_desc(), qsl=FAKE, sl=FAKE, bt=FAKE, bts=64, R=4, T=4, mq=1,
+             ms=1000, scale=0.088, out=FAKE + (1 << 30), lse=None, ws=FAKE + (1 << 32), wsb=1 << 30, opt=None)
+    a.update(kw)
+    return L.pa_attention_decode_fused(a["q"], a["hq"], a["kn"], a["vn"], a["stride"], a["k"], a["v"],
+                                       ctypes.byref(a["desc"]), a["qsl"], a["sl"], a["bt"], a["bts"], a["R"], a["T"],
+                                       a["mq"], a["ms"], ctypes.c_float(a["scale"]), a["out"], a["lse"], a["ws"],
+                                       a["wsb"], a["opt"], None)
+
+
+def test_fused_decode_host_validation(L):
+    assert _fused(L, R=0) == 0
+    assert _fused(L, mq=3) == 2                          # G = 4: 12 rows > the default 8 decode rows
+    o = api.AttnOptions()
+    o.decode_max_query_len = 3
+    # 12 rows allowed with the option: passes validation, then fails only at the (absent) driver
+    assert _fused(L, mq=3, opt=ctypes.byref(o)) in (0, 4)
+    assert _fused(L, kn=None) == 1
+    assert _fused(L, stride=1000) == 1                   # < Hkv * D
+    assert _fused(L, stride=1028) == 2                   # not a multiple of 8 elements
+    assert _fused(L, kn=FAKE + (1 << 33) + 2) == 2       # k_new not 16-byte aligned
+    assert _fused(L, hq=8 * 3) == 2

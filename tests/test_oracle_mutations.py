@@ -32,6 +32,12 @@ MUTATIONS = [
      "int64_t dst = ((blk * num_kv_heads + (num_kv_heads - 1 - h)) * block_size + off) * head_dim;",
      ["kv_write", "slots"]),
     ("lse_missing_max", "*lse = mx + log(z);", "*lse = log(z);", ["brute", "two_key"]),
+    ("pack_k_and_v_swapped", "memcpy(dk, k_cache + b * block_elems,", "memcpy(dk, v_cache + b * block_elems,",
+     ["pack"]),
+    ("pack_block_off_by_one", "memcpy(dv, v_cache + b * block_elems,", "memcpy(dv, v_cache + (b + 1) % num_blocks * block_elems,",
+     ["pack"]),
+    ("unpack_wrong_entry", "memcpy(k_cache + b * block_elems, staging + (2 * i) * block_elems,",
+     "memcpy(k_cache + b * block_elems, staging + (2 * (n - 1 - i)) * block_elems,", ["unpack"]),
 ]
 
 CHECKS = {
@@ -42,6 +48,8 @@ CHECKS = {
     "slots": lambda: pins.test_slot_mapping_matches_allocator_and_round_trips_through_gather(),
     "gather": lambda: pins.test_gather_walks_blocks_in_table_order(),
     "kv_write": lambda: pins.test_kv_write_byte_exact_and_preserves_untouched_slots(),
+    "pack": lambda: pins.test_kv_pack_matches_brute_force_and_the_gather(),
+    "unpack": lambda: pins.test_kv_unpack_inverts_pack_and_touches_nothing_else(),
 }
 
 

@@ -369,3 +369,61 @@ def test_gather_walks_blocks_in_table_order():
     out = oracle.gather_kv(cache, bt, L)
     for j in range(L):
         assert np.array_equal(out[j], cache[bt[j // 16], :, j % 16])
+
+
+# ----------------------------------------------------------------------------
+# block pack / unpack (KV transfer between a prefill and a decode instance)
+# ----------------------------------------------------------------------------
+
+def _brute_pack(k_cache, v_cache, ids):
+    """Pure-Python pack: entry i = the block's values in memory order, K then V."""
+    NB = k_cache.shape[0]
+    flat_k = k_cache.reshape(NB, -1).tolist()
+    flat_v = v_cache.reshape(NB, -1).tolist()
+    elems = len(flat_k[0])
+    out = []
+    for b in ids.tolist():
+        if 0 <= b < NB:
+            out.append([flat_k[b], flat_v[b]])
+        else:
+            out.append([[0] * elems, [0] * elems])
+    return np.array(out, dtype=np.uint16).reshape(len(ids), 2, elems)
+
+
+def test_kv_pack_matches_brute_force_and_the_gather():
+    rng = np.random.default_rng(77)
+    NB, Hkv, D = 12, 3, 8
+    k = rng.integers(0, 1 << 16, size=(NB, Hkv, 16, D), dtype=np.uint16)
+    v = rng.integers(0, 1 << 16, size=(NB, Hkv, 16, D), dtype=np.uint16)
+    ids = np.array([7, 2, 11, 0, 5], np.int32)
+    st = oracle.kv_pack(k, v, ids)
+    assert np.array_equal(st, _brute_pack(k, v, ids))
+    # the packed K/V of a request whose table is `ids` are its gathered tokens, block by block
+    L = 16 * len(ids)
+    for c, cache in ((0, k), (1, v)):
+        g = oracle.gather_kv(cache, ids, L)                              # [L, Hkv, D]
+        packed = st[:, c].reshape(len(ids), Hkv, 16, D).transpose(0, 2, 1, 3).reshape(L, Hkv, D)
+        assert np.array_equal(packed, g)
+    # ids outside the pool pack zeros
+    st2 = oracle.kv_pack(k, v, np.array([3, -1, NB], np.int32))
+    assert np.array_equal(st2[0], st[0] * 0 + np.stack([k[3].reshape(-1), v[3].reshape(-1)]))
+    assert not st2[1:].any()
+
+
+def test_kv_unpack_inverts_pack_and_touches_nothing_else():
+    rng = np.random.default_rng(78)
+    NB, Hkv, D = 10, 2, 8
+    k = rng.integers(0, 1 << 16, size=(NB, 16, Hkv, D), dtype=np.uint16)   # any layout: whole blocks move
+    v = rng.integers(0, 1 << 16, size=(NB, 16, Hkv, D), dtype=np.uint16)
+    src = np.array([1, 8, 4], np.int32)
+    dst = np.array([9, 0, 3], np.int32)
+    st = oracle.kv_pack(k, v, src)
+    fill = np.full_like(k, W.BF16_QNAN)
+    k2, v2 = oracle.kv_unpack(st, dst, fill, fill)
+    for a, b in zip(src, dst):
+        assert np.array_equal(k2[b], k[a]) and np.array_equal(v2[b], v[a])
+    others = np.setdiff1d(np.arange(NB), dst)
+    assert (k2[others] == W.BF16_QNAN).all() and (v2[others] == W.BF16_QNAN).all()
+    # an id outside the pool is skipped
+    k3, _ = oracle.kv_unpack(st, np.array([2, -5, NB + 1], np.int32), fill, fill)
+    assert np.array_equal(k3[2], k[1]) and (k3[np.arange(NB) != 2] == W.BF16_QNAN).all()
