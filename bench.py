@@ -395,6 +395,38 @@ def _follow_on(st: Step, steps: int, warmup: int, peaks: dict):
     return res, launches
 
 
+def _prefix_hash_rate():
+    """Host-side prefix caching on the prefix-sharing workload's shape (128 requests, 2048 shared prompt
+    tokens plus private suffixes, synthetic token ids): chained block hashing of every request and the
+    longest-hit walk of every request after all were inserted.  One host thread."""
+    from paged_kv_cache_461_b200 import api
+    from paged_kv_cache_461_b200 import workloads as W
+    lay = W.workload_layout("prefix_sharing")
+    rng = np.random.default_rng(5)
+    shared = rng.integers(0, 128256, size=2048).astype(np.int32)
+    reqs = [np.concatenate([shared, rng.integers(0, 128256, size=int(L) - 2048).astype(np.int32)])
+            for L in lay.seq_lens]
+    n_tok = sum(len(t) for t in reqs)
+    res = {"requests": len(reqs), "tokens": n_tok, "threads": 1, "where": "host (C++ in libpa_b200.so)"}
+    for algo in ("fnv1a64", "sha256"):
+        t0 = time.perf_counter()
+        hs = [api.prefix_block_hashes(t, algo) for t in reqs]
+        dt = time.perf_counter() - t0
+        res[f"{algo}_tokens_per_s"] = n_tok / dt
+        res[f"{algo}_blocks_per_s"] = sum(len(h) for h in hs) / dt
+    cache = api.PrefixCache()
+    hs = [api.prefix_block_hashes(t) for t in reqs]
+    for r, h in enumerate(hs):
+        cache.insert(h, lay.block_table[r, :len(h)])
+    t0 = time.perf_counter()
+    hits = sum(len(cache.longest_hit(h)) for h in hs)
+    dt = time.perf_counter() - t0
+    res["longest_hit_blocks_per_s"] = hits / dt
+    res["longest_hit_calls_per_s"] = len(hs) / dt
+    cache.close()
+    return res
+
+
 # --------------------------------------------------------------------------- CPU oracle leg
 
 def _oracle_sample(name: str, n_requests: int, seed=None):
@@ -559,6 +591,7 @@ def main():
                        "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
     if not args.no_extras and rank == 0:
         line["follow_on"], n_l = _follow_on(st, max(10, min(args.steps, 50)), args.warmup, peaks)
+        line["follow_on"]["prefix_hash"] = _prefix_hash_rate()
         line["gpu_launches"] += n_l
     if not args.no_extras:
         del st

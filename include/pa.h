@@ -321,6 +321,57 @@ PA_API pa_status_t pa_kv_unpack(const void *staging, const int32_t *block_ids, i
                                 void *v_cache, const pa_cache_desc_t *cache, pa_stream_t stream);
 
 /*
+ * Prefix caching on the host: chained block hashes and the longest cached
+ * prefix.  (shengyayun.com 关键实现细节 item 2: the scheduler hashes each
+ * request in 16-token blocks -- a built-in hash by default, SHA-256 against
+ * collisions -- and find_longest_cache_hit walks the hashes in order through
+ * the map from block hash to cached block, reusing every hit's KV block as it
+ * is; item 1: only whole blocks are reused, a trailing partial block is not.
+ * hn.213312.xyz section 二, item 2.)
+ *
+ * All pointers of these functions are HOST pointers; nothing touches the GPU.
+ *
+ * Block b (tokens 16b .. 16b+15) gets the digest of the byte string
+ *   parent (32 bytes) || its 16 token ids as little-endian int32,
+ * where parent is block b-1's digest, or *root for block 0 (32 zero bytes if
+ * root is NULL; a caller may fold extra keys into it).  Equal digests thus
+ * stand for equal whole prefixes.  PA_HASH_FNV1A64: 64-bit FNV-1a, stored
+ * little-endian in bytes 0..7, bytes 8..31 zero.  PA_HASH_SHA256: SHA-256
+ * (FIPS 180-4), all 32 bytes.
+ */
+#define PA_HASH_FNV1A64 0
+#define PA_HASH_SHA256 1
+typedef struct pa_block_hash {
+    uint8_t bytes[32];
+} pa_block_hash_t;
+
+/* Digests of the num_tokens / 16 full blocks of token_ids (host int32
+ * [num_tokens]) into out_hashes (host, room for num_tokens / 16 entries);
+ * *num_blocks receives that count.  INVALID_ARG on a negative count, a null
+ * pointer that is needed, or an unknown algo. */
+PA_API pa_status_t pa_prefix_block_hashes(const int32_t *token_ids, int64_t num_tokens, const pa_block_hash_t *root,
+                                          int32_t algo, pa_block_hash_t *out_hashes, int64_t *num_blocks);
+
+/* A map from block digest to physical block id, and back (one digest per
+ * block).  Safe to call from several host threads. */
+typedef struct pa_prefix_cache pa_prefix_cache_t;
+PA_API pa_prefix_cache_t *pa_prefix_cache_create(void); /* NULL if out of host memory */
+PA_API void pa_prefix_cache_destroy(pa_prefix_cache_t *cache);
+/* Record that block block_ids[i] holds the KV of the prefix hashes[i] names.
+ * A digest or a block already present keeps its first mapping.  Block ids
+ * must be >= 0 (else INVALID_ARG, nothing recorded). */
+PA_API pa_status_t pa_prefix_cache_insert(pa_prefix_cache_t *cache, const pa_block_hash_t *hashes,
+                                          const int32_t *block_ids, int32_t n);
+/* Forget block_id (when the allocator hands it out for other tokens). */
+PA_API pa_status_t pa_prefix_cache_remove_block(pa_prefix_cache_t *cache, int32_t block_id);
+/* Longest cached prefix: walks hashes[0..n) in order, writes the cached block
+ * of each hit to out_block_ids and stops at the first miss.  Returns the
+ * number of hits, or -1 on invalid arguments. */
+PA_API int32_t pa_prefix_cache_longest_hit(pa_prefix_cache_t *cache, const pa_block_hash_t *hashes, int32_t n,
+                                           int32_t *out_block_ids);
+PA_API int64_t pa_prefix_cache_size(pa_prefix_cache_t *cache); /* digests held, -1 for NULL */
+
+/*
  * pa_debug_gather_kv -- test helper: contiguous copy of one request's first
  * seq_len tokens of a cache, following its block table row (device int32
  * [ceil(seq_len/16)]).  out: bf16 [seq_len, num_kv_heads, head_dim].  A block

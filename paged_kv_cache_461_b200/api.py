@@ -2,7 +2,8 @@
 
 Every function here has the name of a C entry point in include/pa.h minus the
 ``pa_`` prefix, takes torch CUDA tensors, passes their data pointers and the
-current stream to the library, and raises PaError on a non-PA_OK status.
+current stream to the library, and raises PaError on a non-PA_OK status.  The
+prefix-cache functions work on host numpy arrays (they never touch the GPU).
 All arithmetic runs in the library's CUDA kernels; there is no fallback: if
 the library is missing, every call raises.
 """
@@ -28,7 +29,10 @@ DEVICE_WAIT_TIMEOUT = 4
 # every symbol include/pa.h declares
 EXPORTED = ("pa_abi_version", "pa_status_string", "pa_kv_write", "pa_build_slot_mapping", "pa_workspace_size",
             "pa_workspace_size_ex", "pa_attention_mixed", "pa_attention_mixed_ex", "pa_attention_mixed_noalloc",
-            "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack", "pa_merge_attn_states", "pa_debug_gather_kv")
+            "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack", "pa_merge_attn_states", "pa_debug_gather_kv",
+            "pa_prefix_block_hashes", "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_cache_insert",
+            "pa_prefix_cache_remove_block", "pa_prefix_cache_longest_hit", "pa_prefix_cache_size")
+HASH_ALGOS = {"fnv1a64": 0, "sha256": 1}
 LAYOUT_HND = 0   # cache [num_blocks, num_kv_heads, 16, head_dim]
 LAYOUT_NHD = 1   # cache [num_blocks, 16, num_kv_heads, head_dim]
 _LAYOUTS = {"HND": LAYOUT_HND, "NHD": LAYOUT_NHD}
@@ -84,6 +88,20 @@ def lib():
         L.pa_kv_unpack.argtypes = [_vp, _vp, _i32, _vp, _vp, ctypes.POINTER(CacheDesc), _vp]
         L.pa_merge_attn_states.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
         L.pa_debug_gather_kv.argtypes = [_vp, ctypes.POINTER(CacheDesc), _vp, _i32, _vp, _vp]
+        L.pa_prefix_block_hashes.argtypes = [_vp, _i64, _vp, _i32, _vp, ctypes.POINTER(ctypes.c_int64)]
+        L.pa_prefix_block_hashes.restype = ctypes.c_int
+        L.pa_prefix_cache_create.restype = _vp
+        L.pa_prefix_cache_create.argtypes = []
+        L.pa_prefix_cache_destroy.argtypes = [_vp]
+        L.pa_prefix_cache_destroy.restype = None
+        L.pa_prefix_cache_insert.argtypes = [_vp, _vp, _vp, _i32]
+        L.pa_prefix_cache_insert.restype = ctypes.c_int
+        L.pa_prefix_cache_remove_block.argtypes = [_vp, _i32]
+        L.pa_prefix_cache_remove_block.restype = ctypes.c_int
+        L.pa_prefix_cache_longest_hit.argtypes = [_vp, _vp, _i32, _vp]
+        L.pa_prefix_cache_longest_hit.restype = _i32
+        L.pa_prefix_cache_size.argtypes = [_vp]
+        L.pa_prefix_cache_size.restype = _i64
         for name in ("pa_kv_write", "pa_build_slot_mapping", "pa_attention_mixed", "pa_attention_mixed_ex",
                      "pa_attention_mixed_noalloc", "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack",
                      "pa_merge_attn_states", "pa_debug_gather_kv"):
@@ -307,6 +325,71 @@ def debug_gather_kv(cache: torch.Tensor, bt_row: torch.Tensor, seq_len: int, str
     _check(lib().pa_debug_gather_kv(_ptr(cache), ctypes.byref(d), _ptr(bt_row), seq_len, _ptr(out),
                                     _stream(stream)), "pa_debug_gather_kv")
     return out
+
+
+# ---------------------------------------------------------------- prefix caching (host side)
+
+def prefix_block_hashes(token_ids, algo: str = "fnv1a64", root: Optional[bytes] = None):
+    """pa_prefix_block_hashes: chained digests of the full 16-token blocks of a host int32 token array,
+    as a numpy uint8 array [len(token_ids) // 16, 32]."""
+    import numpy as np
+    toks = np.ascontiguousarray(token_ids, dtype=np.int32)
+    out = np.zeros((len(toks) // 16, 32), dtype=np.uint8)
+    n = ctypes.c_int64(0)
+    r = None
+    if root is not None:
+        rb = np.frombuffer(bytes(root), dtype=np.uint8)
+        if rb.size != 32:
+            raise ValueError("root digest must be 32 bytes")
+        r = rb.ctypes.data
+    _check(lib().pa_prefix_block_hashes(toks.ctypes.data if len(toks) else None, len(toks), r, HASH_ALGOS[algo],
+                                        out.ctypes.data if len(out) else None, ctypes.byref(n)),
+           "pa_prefix_block_hashes")
+    assert n.value == len(out)
+    return out
+
+
+class PrefixCache:
+    """pa_prefix_cache_*: block digest -> physical block id, with the longest cached prefix lookup."""
+
+    def __init__(self):
+        self._h = lib().pa_prefix_cache_create()
+        if not self._h:
+            raise MemoryError("pa_prefix_cache_create")
+
+    def close(self):
+        if self._h:
+            lib().pa_prefix_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def insert(self, hashes, block_ids) -> None:
+        import numpy as np
+        h = np.ascontiguousarray(hashes, dtype=np.uint8).reshape(-1, 32)
+        b = np.ascontiguousarray(block_ids, dtype=np.int32)
+        assert len(h) == len(b)
+        _check(lib().pa_prefix_cache_insert(self._h, h.ctypes.data, b.ctypes.data, len(b)), "pa_prefix_cache_insert")
+
+    def remove_block(self, block_id: int) -> None:
+        _check(lib().pa_prefix_cache_remove_block(self._h, int(block_id)), "pa_prefix_cache_remove_block")
+
+    def longest_hit(self, hashes):
+        import numpy as np
+        h = np.ascontiguousarray(hashes, dtype=np.uint8).reshape(-1, 32)
+        out = np.zeros(len(h), dtype=np.int32)
+        n = lib().pa_prefix_cache_longest_hit(self._h, h.ctypes.data if len(h) else None, len(h),
+                                              out.ctypes.data if len(h) else None)
+        if n < 0:
+            raise PaError(1, "pa_prefix_cache_longest_hit")
+        return out[:n]
+
+    def __len__(self):
+        return int(lib().pa_prefix_cache_size(self._h))
 
 
 def read_device_status(workspace: torch.Tensor) -> int:

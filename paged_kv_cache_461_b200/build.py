@@ -16,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpa_b200.so")
-SOURCES = ["pa_api.cu", "kv_write.cu", "plan_merge.cu", "decode.cu", "prefill.cu", "pa_noalloc.cu"]
+SOURCES = ["pa_api.cu", "kv_write.cu", "plan_merge.cu", "decode.cu", "prefill.cu", "pa_noalloc.cu", "prefix_cache.cpp"]
 HEADERS = ["ptx.cuh", "tcgen05.cuh", "pa_internal.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
