@@ -260,7 +260,8 @@ def _attention_only_ms(st: Step, steps: int):
 
 
 def _prefill_only(st: Step, steps: int, warmup: int):
-    """Time pa_attention_mixed on the prefill chunks of the mixed step alone."""
+    """Time pa_attention_mixed on the prefill chunks of the mixed step alone, as a prefill-only
+    batch (decode_max_query_len = -1: the prefill kernel alone, no decode grid beside it)."""
     import torch
     from paged_kv_cache_461_b200 import workloads as W
     lay = st.lay
@@ -274,11 +275,13 @@ def _prefill_only(st: Step, steps: int, warmup: int):
     sl_d = torch.from_numpy(sub.seq_lens).cuda()
     bt_d = torch.from_numpy(sub.block_table).cuda()
     out = torch.empty_like(q)
-    ws = st.api.alloc_workspace(sub.num_seqs, sub.num_tokens, sub.num_q_heads, st.vals.k_cache, sub.max_seq_len)
+    ws = st.api.alloc_workspace(sub.num_seqs, sub.num_tokens, sub.num_q_heads, st.vals.k_cache, sub.max_seq_len,
+                                decode_max_query_len=-1)
 
     def call():
         st.api.attention_mixed(q, st.vals.k_cache, st.vals.v_cache, qsl_d, sl_d, bt_d, sub.max_query_len,
-                               sub.max_seq_len, softmax_scale=st.scale, out=out, workspace=ws)
+                               sub.max_seq_len, softmax_scale=st.scale, out=out, workspace=ws,
+                               decode_max_query_len=-1)
     for _ in range(warmup):
         call()
     torch.cuda.synchronize()
@@ -391,6 +394,37 @@ def _follow_on(st: Step, steps: int, warmup: int, peaks: dict):
                         "blocks": len(ids), "bytes_read_plus_written": moved}
     res["peak"] = {"hbm_gbs": hbm, "source": f"{peaks['source']} hbm_gbs (burst copy)"}
     del staging
+    torch.cuda.empty_cache()
+
+    # speculative verification: the same requests, each scoring k = 3 drafted tokens plus the last
+    # accepted one (q_len 4, 16 packed rows per kv head) in one pass
+    from paged_kv_cache_461_b200 import workloads as W
+    sl = W.build_layout("spec_verify_k3", lay.ctx_lens, np.full(lay.num_seqs, 4, np.int32),
+                        num_q_heads=lay.num_q_heads, num_kv_heads=lay.num_kv_heads, head_dim=lay.head_dim,
+                        num_blocks=lay.num_blocks, seed=lay.seed)
+    sv = W.make_values_torch(sl, "cuda")
+    sq = {k: torch.from_numpy(a).cuda() for k, a in (("qsl", sl.query_start_loc), ("sl", sl.seq_lens),
+                                                       ("bt", sl.block_table), ("slots", sl.slot_mapping))}
+    api.kv_write(sv.k_new, sv.v_new, sq["slots"], sv.k_cache, sv.v_cache)
+    s_out = torch.empty_like(sv.q)
+    ws_dec = api.alloc_workspace(sl.num_seqs, sl.num_tokens, sl.num_q_heads, sv.k_cache, sl.max_seq_len,
+                                 decode_max_query_len=4)
+    ws_pf = api.alloc_workspace(sl.num_seqs, sl.num_tokens, sl.num_q_heads, sv.k_cache, sl.max_seq_len)
+
+    def spec(dq, wsp):
+        return lambda: api.attention_mixed(sv.q, sv.k_cache, sv.v_cache, sq["qsl"], sq["sl"], sq["bt"],
+                                           sl.max_query_len, sl.max_seq_len, out=s_out, workspace=wsp,
+                                           decode_max_query_len=dq)
+    ms_dec = _time_region(spec(4, ws_dec), steps, warmup, 1) / steps
+    ms_pf = _time_region(spec(0, ws_pf), steps, warmup, 1) / steps
+    launches += 7 * steps  # plan+decode+reduce; plan+decode+reduce (no work)+prefill
+    kvb = sl.kv_bytes()
+    res["spec_verify_k3"] = {"value": kvb / (ms_dec * 1e-3) / 1e9, "unit": "GB/s",
+                             "frac": kvb / (ms_dec * 1e-3) / 1e9 / hbm, "ms_per_launch": ms_dec,
+                             "tokens_per_s": sl.num_tokens / (ms_dec * 1e-3),
+                             "ms_per_launch_through_prefill_kernel": ms_pf,
+                             "workload": {**sl.describe(), "q_len": 4, "decode_max_query_len": 4}}
+    del sv, s_out, ws_dec, ws_pf
     torch.cuda.empty_cache()
     return res, launches
 
@@ -607,7 +641,7 @@ def main():
             "prefill_flops_per_step": mx.prefill_flops,
             "prefill_roofline": {"bound": "tensor", "achieved": pf_tf, "peak": peaks["bf16_tflops"],
                                  "unit": "TFLOP/s", "frac": pf_tf / peaks["bf16_tflops"], "ms_per_launch": pf_ms,
-                                 "kernel": "pa_attention_mixed on the prefill chunks alone (prefill_kernel)",
+                                 "kernel": "pa_attention_mixed on the prefill chunks alone, prefill-only mode (plan + prefill_kernel)",
                                  "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                                  "clocks": pf_clocks}}
         line["gpu_launches"] += mx.launches_per_step * mk

@@ -22,8 +22,10 @@
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; only the
  *     pa_cache_desc_t / pa_attn_options_t structs are read from host memory,
- *     during the call.  The library never allocates, frees or synchronises:
- *     work is enqueued on `stream` and the call returns at once.
+ *     during the call (the prefix-cache functions are host-only, see there).
+ *     The library never allocates device memory, frees or synchronises: work
+ *     is enqueued on `stream` and the call returns at once (mixed steps also
+ *     use one library-owned side stream, see pa_attention_mixed).
  *   - bf16 tensors are IEEE bfloat16 (2 bytes per element).
  *   - Host-side validation happens before anything is enqueued; a non-PA_OK
  *     status means nothing was enqueued, except PA_ERR_CUDA (a launch failed).
@@ -90,7 +92,11 @@ typedef struct pa_attn_options {
                                       (shengyayun.com 关键实现细节 3: the target model checks the
                                       k candidates in one pass); 0 = default (8 / G query rows,
                                       at least 1).  Allowed up to 16 / G (G = num_q_heads /
-                                      num_kv_heads), else PA_ERR_UNSUPPORTED. */
+                                      num_kv_heads), else PA_ERR_UNSUPPORTED.  -1: no decode
+                                      kernel, every request takes the prefill kernel -- for
+                                      batches known to hold only prefill work (a prefill
+                                      instance under prefill/decode disaggregation); such a
+                                      call never runs a decode grid beside prefill. */
     int32_t reserved[6];           /* must be zero */
 } pa_attn_options_t;
 
@@ -189,6 +195,16 @@ PA_API size_t pa_workspace_size_ex(int32_t num_seqs, int32_t num_tokens, int32_t
  * divisor of 128.  Errors: INVALID_ARG (null pointer, negative size,
  * num_q_heads % num_kv_heads != 0, bt_stride too small, out overlapping q,
  * nonzero reserved option), UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA.
+ *
+ * Concurrency inside a call: when a step can hold both prefill-shaped and
+ * decode-shaped requests, the prefill kernel runs on a side stream of the
+ * library, beside the decode kernel on `stream`, on an SM share the device
+ * plan picks; `stream` waits for it before the call's work is complete (an
+ * event fork/join, so the call is still one ordered unit on `stream` and can
+ * be captured into a CUDA graph).  The side stream and its two events are
+ * created on the first such call on a device and kept for the process; make
+ * that first call outside stream capture.  This is the only resource the
+ * library creates on its own.
  */
 PA_API pa_status_t pa_attention_mixed(const void *q, int32_t num_q_heads, const void *k_cache,
                                const void *v_cache, const pa_cache_desc_t *cache,

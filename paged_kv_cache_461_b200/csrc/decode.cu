@@ -459,7 +459,7 @@ cudaError_t launch_decode_t(const AttnParams &p, const CUtensorMap &tk, const CU
 } // namespace
 
 cudaError_t launch_decode(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int NT,
-                          int64_t grid_units, int /*num_sms*/, cudaStream_t s)
+                          int64_t grid_units, cudaStream_t s)
 {
     if (grid_units <= 0)
         return cudaSuccess;

@@ -69,11 +69,15 @@ bool make_plan(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, const 
     }
     // decode path: up to 8*NT packed (token, head) rows per kv head in one warp MMA
     const int dq = o ? o->decode_max_query_len : 0;
-    if (dq < 0 || (dq > 0 && dq * P.G > 16)) {
-        *why = dq < 0 ? PA_ERR_INVALID_ARG : PA_ERR_UNSUPPORTED;
+    if (dq < -1 || (dq > 0 && dq * P.G > 16)) {
+        *why = dq < -1 ? PA_ERR_INVALID_ARG : PA_ERR_UNSUPPORTED;
         return false;
     }
-    if (dq > 0) {
+    if (dq == -1) { // no decode kernel: every request takes the prefill kernel
+        P.NT = 0;
+        P.QD = 0;
+        P.dec_rows_cap = 0;
+    } else if (dq > 0) {
         P.NT = dq * P.G <= 8 ? 1 : 2;
         P.QD = dq;
         P.dec_rows_cap = dq * P.G;
@@ -193,6 +197,37 @@ int device_sms()
 }
 
 pa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+// Per-device side stream and fork/join events for running the prefill kernel beside the
+// decode kernel of the same step.  Created on the first mixed call on a device and kept for
+// the life of the process.  The mutex orders the host-side record/wait pairs of concurrent
+// callers (the events are shared).
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex mu;
+    bool ready = false;
+};
+
+SideStream *side_stream()
+{
+    static SideStream table[64];
+    static std::mutex init_mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    SideStream &ss = table[dev];
+    std::lock_guard<std::mutex> g(init_mu);
+    if (!ss.ready) {
+        if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess)
+            return nullptr;
+        if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+            return nullptr;
+        ss.ready = true;
+    }
+    return &ss;
+}
 
 } // namespace
 
@@ -366,11 +401,36 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     }
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    p.num_sms = device_sms();
+    const bool prefill = (int64_t)max_query_len * P.G > P.dec_rows_cap;
+    CUtensorMap tq;
+    if (prefill && !get_map(q, 3, D, (uint64_t)num_q_heads, (uint64_t)num_tokens, (uint32_t)P.G,
+                            (uint32_t)(kPrefillRows / P.G), &tq))
+        return PA_ERR_CUDA;
+    // A mixed step forks after the plan: prefill (persistent, on the plan's share of the SMs, at
+    // the highest priority) on the side stream, decode and the split-KV reduce on the caller's
+    // stream, which then waits for prefill.  The two kernels never touch the same output rows.
+    SideStream *ss = (prefill && P.NT > 0) ? side_stream() : nullptr;
+    if (prefill && P.NT > 0 && !ss)
+        return PA_ERR_CUDA;
     cudaError_t e = launch_plan(p, s);
     if (e != cudaSuccess)
         return PA_ERR_CUDA;
+    std::unique_lock<std::mutex> fork_lock;
+    if (ss) {
+        fork_lock = std::unique_lock<std::mutex>(ss->mu);
+        if (cudaEventRecord(ss->fork, s) != cudaSuccess || cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+            return PA_ERR_CUDA;
+    }
+    if (prefill) {
+        e = launch_prefill(p, tq, tk, tv, P.max_pf_tiles, p.num_sms, ss ? ss->stream : s);
+        if (e != cudaSuccess)
+            return PA_ERR_CUDA;
+    }
+    if (ss && cudaEventRecord(ss->join, ss->stream) != cudaSuccess)
+        return PA_ERR_CUDA;
     if (P.NT > 0) {
-        e = launch_decode(p, tk, tv, P.NT, P.max_dec_units, device_sms(), s);
+        e = launch_decode(p, tk, tv, P.NT, P.max_dec_units, s);
         if (e != cudaSuccess)
             return PA_ERR_CUDA;
         if (P.need_reduce) {
@@ -379,15 +439,8 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
                 return PA_ERR_CUDA;
         }
     }
-    if ((int64_t)max_query_len * P.G > P.dec_rows_cap) {
-        CUtensorMap tq;
-        if (!get_map(q, 3, D, (uint64_t)num_q_heads, (uint64_t)num_tokens, (uint32_t)P.G,
-                     (uint32_t)(kPrefillRows / P.G), &tq))
-            return PA_ERR_CUDA;
-        e = launch_prefill(p, tq, tk, tv, P.max_pf_tiles, device_sms(), s);
-        if (e != cudaSuccess)
-            return PA_ERR_CUDA;
-    }
+    if (ss && cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
+        return PA_ERR_CUDA;
     return PA_OK;
 }
 

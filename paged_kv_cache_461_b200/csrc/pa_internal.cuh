@@ -23,7 +23,8 @@ struct WsHeader {
     uint32_t n_dec_units; // (request, split) decode work items
     uint32_t n_pf_tiles;  // (request, q-tile) prefill work items
     uint32_t n_reduce;    // decode requests with more than one split
-    uint32_t pad[60];
+    uint32_t pf_ctas;     // persistent prefill CTAs that take work; the others leave their SM to decode
+    uint32_t pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -65,6 +66,7 @@ struct AttnParams {
     float *part_lse;            // [num_seqs*QD*Hq*max_splits]
     int split_tokens, max_splits, QD, dec_rows_cap;
     int nhd;                    // cache layout PA_LAYOUT_NHD (else HND)
+    int num_sms;                // SMs of the device (the plan splits them between prefill and decode)
     // fused KV write (pa_attention_decode_fused); k_new == nullptr otherwise
     const uint16_t *k_new, *v_new;
     int64_t new_row_stride;     // elements
@@ -85,7 +87,7 @@ cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D,
                           int seq_len, void *out, cudaStream_t s);
 cudaError_t launch_plan(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_decode(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int NT,
-                          int64_t grid_units, int num_sms, cudaStream_t s);
+                          int64_t grid_units, cudaStream_t s);
 cudaError_t launch_reduce(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_merge_states(const float *part_out, const float *part_lse, const int32_t *parts_per_row,
                                 int num_rows, int num_heads, int num_parts, int D, void *out, float *lse_out,

@@ -69,6 +69,56 @@ __device__ __forceinline__ void cta_excl_scan3(int a, int b, int c, int &ea, int
     __syncthreads();
 }
 
+// SM split of a mixed step.  The prefill kernel (tensor bound) and the decode kernel (HBM
+// bound) run at the same time on disjoint SMs: the plan keeps pf_ctas persistent prefill CTAs
+// busy and the decode CTAs take every other SM, and all of them once prefill is done.  Rates
+// measured on B200 with this library's kernels running side by side (power-capped clocks):
+//   prefill  ~5.6 TFLOP/s per SM;
+//   decode   ~65 GB/s per SM (two CTAs, ~190 KB of loads in flight per SM, so latency
+//            bound when confined to part of the GPU), at most the HBM rate.
+constexpr float kPfFlopsPerSm = 5.6e12f;
+constexpr float kDecBytesPerSm = 65e9f;
+constexpr float kDecBytesMax = 6.35e12f;
+
+// Modelled step time (seconds) with pp prefill SMs out of num_sms: prefill lasts F / (pp f);
+// decode runs at min(B, (S - pp) b) meanwhile and at B after that.
+__device__ __forceinline__ float split_time(float pf_flops, float dec_bytes, int num_sms, int pp)
+{
+    const float t_pf = pf_flops / ((float)pp * kPfFlopsPerSm);
+    const float r_dec = fminf(kDecBytesMax, (float)(num_sms - pp) * kDecBytesPerSm);
+    const float done = r_dec * t_pf;
+    return done >= dec_bytes ? t_pf : t_pf + (dec_bytes - done) / kDecBytesMax;
+}
+
+// Prefill CTAs that minimise the modelled step time: every thread of the CTA evaluates one
+// candidate, then a block-wide argmin (ties go to the larger count).  Called by all threads.
+__device__ int choose_pf_ctas(float pf_flops, float dec_bytes, int num_sms, int pf_items)
+{
+    __shared__ unsigned long long s_best[32];
+    const int cap = max(1, min(num_sms, pf_items));
+    if (pf_flops <= 0.f || dec_bytes <= 0.f)
+        return cap;
+    // key = (time bits, cap - pp): time is non-negative, so its float bits order like the value
+    unsigned long long key = ~0ull;
+    for (int pp = (int)threadIdx.x + 1; pp <= cap; pp += blockDim.x) {
+        const float t = split_time(pf_flops, dec_bytes, num_sms, pp);
+        const unsigned long long k = (unsigned long long)__float_as_uint(t) << 32 | (unsigned)(cap - pp);
+        key = k < key ? k : key;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+        key = other < key ? other : key;
+    }
+    if ((threadIdx.x & 31) == 0)
+        s_best[threadIdx.x >> 5] = key;
+    __syncthreads();
+    unsigned long long best = ~0ull;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w)
+        best = s_best[w] < best ? s_best[w] : best;
+    return cap - (int)(best & 0xffffffffu);
+}
+
 // 128-key steps a prefill q-pair of request r needs: keys 0 .. position of its last token
 __device__ __forceinline__ int pair_cost(int ctx, int q_len, int qp, int tq)
 {
@@ -84,9 +134,13 @@ __device__ __forceinline__ int pair_cost(int ctx, int q_len, int qp, int tq)
 __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_buckets)
 {
     extern __shared__ int hist[]; // [n_buckets] pair counts, then start offsets
+    __shared__ unsigned long long s_sum[2][32];
     WsHeader *hdr = p.hdr;
     if (threadIdx.x == 0)
         hdr->status = 0u;
+    // work estimates, per thread then reduced once: keys read by its decode requests and
+    // causal (query, key) pairs of its prefill requests
+    unsigned long long my_dec_tokens = 0ull, my_pf_pairs = 0ull;
     for (int i = threadIdx.x; i < n_buckets; i += blockDim.x)
         hist[i] = 0;
     __syncthreads();
@@ -123,6 +177,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
         classify(r, n_dec, n_pf, red, ctx, q_len);
         for (int k = 0; k < n_pf; ++k)
             atomicAdd(&hist[min(pair_cost(ctx, q_len, k, tq), n_buckets - 1)], 1);
+        if (n_dec)
+            my_dec_tokens += (unsigned long long)(ctx + q_len);
+        if (n_pf)
+            my_pf_pairs += (unsigned long long)q_len * ctx + (unsigned long long)q_len * (q_len + 1) / 2;
         int ed, ep, er, td, tp, tr;
         cta_excl_scan3(n_dec, n_pf, red, ed, ep, er, td, tp, tr);
         for (int s = 0; s < n_dec; ++s)
@@ -156,10 +214,34 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
             p.pf_tiles[pos] = make_int2(r, k);
         }
     }
+    // block sums of the two estimates (warp shuffles, then one warp over the warp partials)
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        my_dec_tokens += __shfl_xor_sync(0xffffffffu, my_dec_tokens, o);
+        my_pf_pairs += __shfl_xor_sync(0xffffffffu, my_pf_pairs, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        s_sum[0][threadIdx.x >> 5] = my_dec_tokens;
+        s_sum[1][threadIdx.x >> 5] = my_pf_pairs;
+    }
+    __syncthreads();
+    unsigned long long dec_tokens = 0ull, pf_pairs = 0ull;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        dec_tokens += s_sum[0][w];
+        pf_pairs += s_sum[1][w];
+    }
+    const float dec_bytes = (float)dec_tokens * (float)(p.Hkv * p.D * 4); // K + V, bf16
+    const float pf_flops = (float)pf_pairs * (float)(4 * p.Hq * p.D);
+    const int pf_ctas = choose_pf_ctas(pf_flops, dec_bytes, p.num_sms, carry_pf * p.Hkv);
     if (threadIdx.x == 0) {
         hdr->n_dec_units = (uint32_t)carry_dec;
         hdr->n_pf_tiles = (uint32_t)carry_pf;
         hdr->n_reduce = (uint32_t)carry_red;
+#ifdef PA_FORCE_PF_CTAS
+        hdr->pf_ctas = (uint32_t)min(PA_FORCE_PF_CTAS, p.num_sms);
+#else
+        hdr->pf_ctas = (uint32_t)pf_ctas;
+#endif
     }
 }
 

@@ -150,11 +150,12 @@ __device__ __forceinline__ ItemGeo item_geo(const AttnParams &p, int item)
 
 // The k-th work item of this CTA.  The work list is sorted by cost, most expensive
 // first; walking it in snake order (CTA b takes item b of even rounds and item
-// grid-1-b of odd rounds) pairs heavy with light items, so the CTAs finish together.
-__device__ __forceinline__ int snake_item(int k)
+// n-1-b of odd rounds, n working CTAs) pairs heavy with light items, so the CTAs
+// finish together.
+__device__ __forceinline__ int snake_item(int k, int n_ctas)
 {
-    const int b = (k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
-    return k * (int)gridDim.x + b;
+    const int b = (k & 1) ? n_ctas - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    return k * n_ctas + b;
 }
 
 __device__ __forceinline__ int blocks_in_step(int n_keys, int j)
@@ -171,8 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     using Cfg = PfCfg<D>;
     constexpr int kKS = D / 16; // k-steps of Q K^T
     const int n_items = (int)p.hdr->n_pf_tiles * p.Hkv;
-    if ((int)blockIdx.x >= n_items || (p.hdr->status & PA_DEVICE_WAIT_TIMEOUT))
-        return; // no work for this CTA, or an earlier CTA of this call already gave up
+    // CTAs that take work: the plan's share of the SMs for prefill (the rest go to decode)
+    const int n_ctas = min(min((int)gridDim.x, n_items), max(1, (int)p.hdr->pf_ctas));
+    if ((int)blockIdx.x >= n_ctas || (p.hdr->status & PA_DEVICE_WAIT_TIMEOUT))
+        return; // no work for this CTA (its SM is left to decode), or an earlier CTA gave up
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         bool ok = true;
         uint32_t gs = 0; // K/V steps loaded so far by this CTA
         uint32_t nq = 0; // items whose Q was loaded
-        for (int k = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++k)) {
+        for (int k = 0, item = snake_item(0, n_ctas); ok && item < n_items; item = snake_item(++k, n_ctas)) {
             const ItemGeo g = item_geo(p, item);
             // Q of this item, once the previous item's last QK^T has read the old Q
             if (nq > 0 && !mbar_wait_warp(bar + B_QE * 8, (nq - 1) & 1, abort_flag)) {
@@ -370,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             uint32_t nfix = 0;          // items with a zeroed V tail
             uint32_t tstep[2] = {0, 0}; // steps of tile X so far (phase of B_SF / B_PF)
             uint32_t titem[2] = {0, 0}; // items with tile X so far (phase of B_OF / B_OE)
-            for (int k = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++k)) {
+            for (int k = 0, item = snake_item(0, n_ctas); ok && item < n_items; item = snake_item(++k, n_ctas)) {
                 const ItemGeo g = item_geo(p, item);
                 const int nkt[2] = {g.t0.nkt, g.t1.nkt};
                 const int pmax[2] = {g.t0.p_max, g.t1.p_max};
@@ -473,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const float thresh = 8.f / c; // 2^8 growth, in raw score units
         bool ok = true;
         uint32_t tstep = 0, titem = 0;
-        for (int k = 0, item = snake_item(0); ok && item < n_items; item = snake_item(++k)) {
+        for (int k = 0, item = snake_item(0, n_ctas); ok && item < n_items; item = snake_item(++k, n_ctas)) {
             const ItemGeo gi = item_geo(p, item);
             const TileGeo g = x ? gi.t1 : gi.t0;
             if (g.rows == 0)
@@ -640,8 +643,22 @@ cudaError_t launch_prefill_t(const AttnParams &p, const CUtensorMap &tq, const C
     // persistent: one CTA per SM, never more CTAs than the largest possible number of items
     const int64_t items = grid_tiles * p.Hkv;
     const unsigned grid = (unsigned)(items < num_sms ? items : num_sms);
-    prefill_kernel<D><<<grid, kThreads, smem, s>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    // launched at the device's highest priority: when the decode kernel of the same step runs
+    // beside it on another stream, the persistent prefill CTAs are placed first and decode
+    // fills the SMs they leave
+    int lo = 0, hi = 0;
+    cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributePriority;
+    attr[0].val.priority = hi;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<D>, tq, tk, tv, p);
 }
 
 } // namespace

@@ -85,8 +85,11 @@ def test_workspace_size_rules(L):
     assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) > 0
     o.decode_max_query_len = 5                      # 20 rows
     assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) == 0
-    o.decode_max_query_len = -1
+    o.decode_max_query_len = -2
     assert L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 1000, ctypes.byref(o)) == 0
+    o.decode_max_query_len = -1                     # prefill kernel only: no split partials needed
+    assert 0 < L.pa_workspace_size_ex(4, 4, 32, ctypes.byref(d), 100000, ctypes.byref(o)) < \
+        L.pa_workspace_size(4, 4, 32, ctypes.byref(d), 100000)
 
 
 FAKE = 1 << 40  # a non-null pointer value; never dereferenced by host validation paths below

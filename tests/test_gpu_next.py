@@ -211,3 +211,33 @@ def test_pack_full_size_request_blocks_sampled():
     torch.cuda.synchronize()
     assert _bits_equal(k2[ids_d.long()], vals.k_cache[ids_d.long()])
     assert _bits_equal(v2[ids_d.long()], vals.v_cache[ids_d.long()])
+
+
+# ----------------------------------------------------------------------------- CUDA graph capture
+
+@pytest.mark.parametrize("kind", ["mixed", "decode"])
+def test_step_replays_from_a_cuda_graph_bit_identically(kind):
+    # a mixed step forks prefill onto the library's side stream and joins it back: the whole call
+    # must still capture into one graph and replay to the same bits as the eager call
+    rng = np.random.default_rng(31)
+    if kind == "mixed":
+        ctx = list(rng.integers(0, 2000, size=20)) + [0, 700, 1500]
+        q = [1] * 20 + [300, 129, 64]
+    else:
+        ctx, q = list(rng.integers(0, 3000, size=40)), [1] * 40
+    lay = _layout("graph", ctx, q, 32, 8, 128, seed=17)
+    st = DevStep(lay, W.make_values_numpy(lay))
+    st.write()
+    out_e, lse_e = st.attend()                       # eager call first (creates the side stream)
+    torch.cuda.synchronize()
+    out_g = torch.full_like(out_e, float("nan"))
+    lse_g = torch.full_like(lse_e, float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        api.attention_mixed(st.q, st.k_cache, st.v_cache, st.qsl, st.seq_lens, st.bt, lay.max_query_len,
+                            lay.max_seq_len, out=out_g, lse=lse_g, workspace=st.workspace)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert _bits_equal(out_g, out_e) and torch.equal(lse_g, lse_e)
+    assert api.read_device_status(st.workspace) == 0

@@ -249,6 +249,35 @@ def test_mixed_step_parity(shuffle):
     lay = _mixed_layout(11, shuffle=shuffle)
     st, out, lse, ref, ref_lse = _run(lay)
     assert_parity(out, ref, lse, ref_lse, what=f"mixed shuffle={shuffle}")
+    # the plan splits the SMs: some persistent prefill CTAs, the rest of the GPU for decode
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n_dec, n_pf, _ = work_counts(st.workspace)
+    pf_ctas = st.workspace[16:20].view(torch.int32).item()
+    assert n_dec > 0 and n_pf > 0 and 1 <= pf_ctas < sms
+
+
+def test_prefill_only_mode_routes_every_request_to_the_prefill_kernel():
+    # decode_max_query_len = -1: decode-shaped requests (q_len 1..2) go through the tensor-core kernel
+    lay = _mixed_layout(13, n_dec=12)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    out, lse = st.attend(decode_max_query_len=-1)
+    torch.cuda.synchronize()
+    n_dec, n_pf, _ = work_counts(st.workspace)
+    assert n_dec == 0 and n_pf > 0
+    ref, ref_lse, _ = oracle_for_step(lay, vals)
+    assert_parity(out, ref, lse, ref_lse, what="prefill-only mode")
+    assert api.read_device_status(st.workspace) == 0
+
+
+def test_prefill_only_step_keeps_every_sm():
+    lay = _layout("pfonly", [0, 500, 40], [700, 900, 300], 32, 8, 128, seed=21)
+    st, out, lse, ref, ref_lse = _run(lay)
+    assert_parity(out, ref, lse, ref_lse, what="prefill only")
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n_dec, n_pf, _ = work_counts(st.workspace)
+    assert n_dec == 0 and st.workspace[16:20].view(torch.int32).item() == min(sms, n_pf * lay.num_kv_heads)
 
 
 @pytest.mark.parametrize("kind", ["q_x8", "v_mean3", "ctx_1_mod_16"])
