@@ -550,11 +550,13 @@ def profile_case(kind: str, launches: int):
     bt = torch.from_numpy(lay.block_table).cuda()
     slots = torch.from_numpy(lay.slot_mapping).cuda()
     api.kv_write(v.k_new, v.v_new, slots, v.k_cache, v.v_cache)
-    ws = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, v.k_cache, lay.max_seq_len)
+    dq = -1 if kind == "prefill" else 0   # the prefill chunks as a prefill-only batch, as bench.py times them
+    ws = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, v.k_cache, lay.max_seq_len,
+                             decode_max_query_len=dq)
     out = torch.empty_like(v.q)
     for _ in range(1 + launches):
         api.attention_mixed(v.q, v.k_cache, v.v_cache, qsl, sl, bt, lay.max_query_len, lay.max_seq_len,
-                            out=out, workspace=ws)
+                            out=out, workspace=ws, decode_max_query_len=dq)
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": kind, **lay.describe(), "kv_bytes": lay.kv_bytes(),
                       "pool_bytes": 2 * v.k_cache.numel() * 2}))
