@@ -22,15 +22,18 @@
 //     registers with movmatrix (no shared-memory round trip);
 //   * O^T += V^T P^T on mma.sync with V^T fragments from ldmatrix.trans;
 //   * at the end the 4 warps' (m, l, O) are merged through shared memory and
-//     written as bf16 output (single split) or as an fp32 partial state for
-//     the split-KV reduce.
+//     written as bf16 output (single split) or as an fp32 partial state; the
+//     last split CTA of a (request, kv head) to finish -- counted with one
+//     atomic per (request, kv head) -- merges all the splits' states into the
+//     output (flash-decoding's second pass without a second launch).
 // Keys beyond L_r in the last block (unused slots, possibly NaN) are masked by
 // select, and their V rows are zeroed in registers, so 0 * NaN never reaches
 // an accumulator.
 #include <math_constants.h>
 
-#include "ptx.cuh"
+#include "merge.cuh"
 #include "pa_internal.cuh"
+#include "ptx.cuh"
 
 namespace pa {
 namespace {
@@ -367,73 +370,99 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
     constexpr int kEpt = D / kTpr;                 // consecutive elements per thread
     const int n = threadIdx.x / kTpr;
     const int d0 = (threadIdx.x % kTpr) * kEpt;
-    if (n >= rows)
-        return;
-    float M = -CUDART_INF_F;
+    // one query row n (elements d0 .. d0+kEpt-1): merge the 4 warps' states, then write the output
+    // (single split) or this split's partial state
+    auto write_state = [&](int n, int d0) {
+        float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) {
-        const float *ml = reinterpret_cast<const float *>(smem + w * kDecStages * Cfg::kStage) + kRows * kLd;
-        M = fmaxf(M, ml[n]);
-    }
-    float wgt[kDecWarps];
-    float lt = 0.f, lx = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) {
-        const float *ml = reinterpret_cast<const float *>(smem + w * kDecStages * Cfg::kStage) + kRows * kLd;
-        const float mw = ml[n];
-        wgt[w] = (mw == -CUDART_INF_F) ? 0.f : fast_exp2(mw - M);
-        lt += ml[kRows + n] * wgt[w];
-        lx += ml[2 * kRows + n] * wgt[w];
-    }
-    const float inv = lt > 0.f ? 1.f / lt : 0.f;
-    float o[kEpt];
-#pragma unroll
-    for (int i = 0; i < kEpt; ++i)
-        o[i] = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) {
-        const float *cb = reinterpret_cast<const float *>(smem + w * kDecStages * Cfg::kStage) + n * kLd + d0;
-#pragma unroll
-        for (int i = 0; i < kEpt; i += 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(cb + i);
-            o[i] += wgt[w] * v.x;
-            o[i + 1] += wgt[w] * v.y;
-            o[i + 2] += wgt[w] * v.z;
-            o[i + 3] += wgt[w] * v.w;
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float *ml = reinterpret_cast<const float *>(smem + w * kDecStages * Cfg::kStage) + kRows * kLd;
+            M = fmaxf(M, ml[n]);
         }
-    }
-    const float lse = lx > 0.f ? (M + log2f(lx)) * 0.69314718055994531f : -CUDART_INF_F;
-    const int t = qs + n / p.G;
-    const int hq = h * p.G + n % p.G;
-    if (n_splits == 1) {
-        __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D + d0;
-        if constexpr (kEpt % 8 == 0) {
+        float wgt[kDecWarps];
+        float lt = 0.f, lx = 0.f;
 #pragma unroll
-            for (int i = 0; i < kEpt; i += 8) {
-                uint4 v;
-                v.x = pack_bf16x2(o[i] * inv, o[i + 1] * inv);
-                v.y = pack_bf16x2(o[i + 2] * inv, o[i + 3] * inv);
-                v.z = pack_bf16x2(o[i + 4] * inv, o[i + 5] * inv);
-                v.w = pack_bf16x2(o[i + 6] * inv, o[i + 7] * inv);
-                *reinterpret_cast<uint4 *>(dst + i) = v;
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float *ml = reinterpret_cast<const float *>(smem + w * kDecStages * Cfg::kStage) + kRows * kLd;
+            const float mw = ml[n];
+            wgt[w] = (mw == -CUDART_INF_F) ? 0.f : fast_exp2(mw - M);
+            lt += ml[kRows + n] * wgt[w];
+            lx += ml[2 * kRows + n] * wgt[w];
+        }
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        float o[kEpt];
+#pragma unroll
+        for (int i = 0; i < kEpt; ++i)
+            o[i] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float *cb = reinterpret_cast<const float *>(smem + w * kDecStages * Cfg::kStage) + n * kLd + d0;
+#pragma unroll
+            for (int i = 0; i < kEpt; i += 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(cb + i);
+                o[i] += wgt[w] * v.x;
+                o[i + 1] += wgt[w] * v.y;
+                o[i + 2] += wgt[w] * v.z;
+                o[i + 3] += wgt[w] * v.w;
             }
-        } else {
-            static_assert(kEpt == 4, "output vector width");
-            uint2 v;
-            v.x = pack_bf16x2(o[0] * inv, o[1] * inv);
-            v.y = pack_bf16x2(o[2] * inv, o[3] * inv);
-            *reinterpret_cast<uint2 *>(dst) = v;
         }
-        if (p.lse && d0 == 0)
-            p.lse[(int64_t)t * p.Hq + hq] = lse;
-    } else {
-        const int64_t idx = (((int64_t)r * p.QD + n / p.G) * p.Hq + hq) * p.max_splits + split;
-        float *dst = p.part_o + idx * D + d0;
+        const float lse = lx > 0.f ? (M + log2f(lx)) * 0.69314718055994531f : -CUDART_INF_F;
+        const int t = qs + n / p.G;
+        const int hq = h * p.G + n % p.G;
+        if (n_splits == 1) {
+            __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D + d0;
+            if constexpr (kEpt % 8 == 0) {
 #pragma unroll
-        for (int i = 0; i < kEpt; i += 4)
-            *reinterpret_cast<float4 *>(dst + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
-        if (d0 == 0)
-            p.part_lse[idx] = lse;
+                for (int i = 0; i < kEpt; i += 8) {
+                    uint4 v;
+                    v.x = pack_bf16x2(o[i] * inv, o[i + 1] * inv);
+                    v.y = pack_bf16x2(o[i + 2] * inv, o[i + 3] * inv);
+                    v.z = pack_bf16x2(o[i + 4] * inv, o[i + 5] * inv);
+                    v.w = pack_bf16x2(o[i + 6] * inv, o[i + 7] * inv);
+                    *reinterpret_cast<uint4 *>(dst + i) = v;
+                }
+            } else {
+                static_assert(kEpt == 4, "output vector width");
+                uint2 v;
+                v.x = pack_bf16x2(o[0] * inv, o[1] * inv);
+                v.y = pack_bf16x2(o[2] * inv, o[3] * inv);
+                *reinterpret_cast<uint2 *>(dst) = v;
+            }
+            if (p.lse && d0 == 0)
+                p.lse[(int64_t)t * p.Hq + hq] = lse;
+        } else {
+            const int64_t idx = (((int64_t)r * p.QD + n / p.G) * p.Hq + hq) * p.max_splits + split;
+            float *dst = p.part_o + idx * D + d0;
+#pragma unroll
+            for (int i = 0; i < kEpt; i += 4)
+                *reinterpret_cast<float4 *>(dst + i) =
+                    make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+            if (d0 == 0)
+                p.part_lse[idx] = lse;
+        }
+    };
+    if (n < rows)
+        write_state(n, d0);
+    if (n_splits == 1)
+        return;
+    // Split request: the last of its split CTAs for this kv head merges all the splits' states.
+    // Release: every thread's partial stores are made visible before the arrival is counted.
+    __threadfence();
+    __syncthreads();
+    __shared__ int s_last;
+    if (threadIdx.x == 0)
+        s_last = atomicAdd(&p.split_arrivals[(int64_t)r * p.Hkv + h], 1u) == (unsigned)(n_splits - 1);
+    __syncthreads();
+    if (!s_last)
+        return;
+    __threadfence(); // acquire: the other splits' states, read below past L1
+    for (int rr = warp; rr < rows; rr += kDecWarps) {
+        const int t = qs + rr / p.G;
+        const int hq = h * p.G + rr % p.G;
+        const int64_t idx = (((int64_t)r * p.QD + rr / p.G) * p.Hq + hq) * p.max_splits;
+        const int64_t orow = (int64_t)t * p.Hq + hq;
+        merge_one<D, true>(p.part_o + idx * D, D, p.part_lse + idx, 1, n_splits, p.out + orow * D,
+                           p.lse ? p.lse + orow : nullptr);
     }
 }
 

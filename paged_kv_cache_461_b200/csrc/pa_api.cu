@@ -99,7 +99,7 @@ bool make_plan(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, const 
     P.off_pf = off;
     off = align_up(off + sizeof(int2) * (size_t)P.max_pf_tiles);
     P.off_red = off;
-    off = align_up(off + sizeof(int32_t) * (size_t)num_seqs);
+    off = align_up(off + sizeof(uint32_t) * (size_t)num_seqs * (size_t)c->num_kv_heads);
     P.off_part_o = off;
     off = align_up(off + sizeof(float) * (size_t)c->head_dim * (size_t)part_rows);
     P.off_part_lse = off;
@@ -384,7 +384,7 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     p.hdr = reinterpret_cast<WsHeader *>(ws);
     p.dec_units = reinterpret_cast<int2 *>(ws + P.off_dec);
     p.pf_tiles = reinterpret_cast<int2 *>(ws + P.off_pf);
-    p.red_list = reinterpret_cast<int32_t *>(ws + P.off_red);
+    p.split_arrivals = reinterpret_cast<uint32_t *>(ws + P.off_red);
     p.part_o = reinterpret_cast<float *>(ws + P.off_part_o);
     p.part_lse = reinterpret_cast<float *>(ws + P.off_part_lse);
     p.split_tokens = P.split_tokens;
@@ -433,11 +433,7 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
         e = launch_decode(p, tk, tv, P.NT, P.max_dec_units, s);
         if (e != cudaSuccess)
             return PA_ERR_CUDA;
-        if (P.need_reduce) {
-            e = launch_reduce(p, s);
-            if (e != cudaSuccess)
-                return PA_ERR_CUDA;
-        }
+
     }
     if (ss && cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
         return PA_ERR_CUDA;

@@ -22,7 +22,7 @@ struct WsHeader {
     uint32_t status;      // PA_DEVICE_* bits
     uint32_t n_dec_units; // (request, split) decode work items
     uint32_t n_pf_tiles;  // (request, q-tile) prefill work items
-    uint32_t n_reduce;    // decode requests with more than one split
+    uint32_t n_reduce;    // decode requests with more than one split (merged by their last split CTA)
     uint32_t pf_ctas;     // persistent prefill CTAs that take work; the others leave their SM to decode
     uint32_t pad[59];
 };
@@ -61,7 +61,7 @@ struct AttnParams {
     WsHeader *hdr;
     int2 *dec_units;            // (r, split)
     int2 *pf_tiles;             // (r, q-tile)
-    int32_t *red_list;          // r
+    uint32_t *split_arrivals;   // [num_seqs * Hkv] split CTAs of (request, kv head) done so far
     float *part_o;              // [num_seqs*QD*Hq*max_splits, D]
     float *part_lse;            // [num_seqs*QD*Hq*max_splits]
     int split_tokens, max_splits, QD, dec_rows_cap;
@@ -88,7 +88,6 @@ cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D,
 cudaError_t launch_plan(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_decode(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int NT,
                           int64_t grid_units, cudaStream_t s);
-cudaError_t launch_reduce(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_merge_states(const float *part_out, const float *part_lse, const int32_t *parts_per_row,
                                 int num_rows, int num_heads, int num_parts, int D, void *out, float *lse_out,
                                 cudaStream_t s);

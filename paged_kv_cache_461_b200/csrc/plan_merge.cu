@@ -9,12 +9,13 @@
 // decodes first and prefill chunks after them (hn.213312.xyz section 一,
 // "调度器"), but nothing here depends on that order.
 //
-// Merge: for each (row, head) with parts s = 0..S-1 holding normalised
-// outputs o_s and natural-log LSEs, LSE = ln sum exp(lse_s) and
-// out = sum exp(lse_s - LSE) o_s -- the flash-decoding second pass, one warp
-// per (row, head), fp32 throughout, bf16 output.
+// pa_merge_attn_states: the merge of attention states (merge.cuh) as a stand-alone call.
+// Inside a step the split-KV merge runs at the end of the decode kernel itself.
 #include <math_constants.h>
 
+#include <type_traits>
+
+#include "merge.cuh"
 #include "pa_internal.cuh"
 
 namespace pa {
@@ -186,7 +187,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
         for (int s = 0; s < n_dec; ++s)
             p.dec_units[carry_dec + ed + s] = make_int2(r, s);
         if (red)
-            p.red_list[carry_red + er] = r;
+            for (int h = 0; h < p.Hkv; ++h)
+                p.split_arrivals[(int64_t)r * p.Hkv + h] = 0u; // counted by the decode kernel
         carry_dec += td;
         carry_pf += tp;
         carry_red += tr;
@@ -245,88 +247,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
     }
 }
 
-// One warp merges the n parts of one (row, head).  o points at part 0's D
-// floats (parts o_stride floats apart), lse at part 0 (lse_stride apart).
-template <int D>
-__device__ __forceinline__ void merge_one(const float *__restrict__ o, int64_t o_stride, const float *__restrict__ lse,
-                                          int lse_stride, int n, __nv_bfloat16 *__restrict__ out, float *lse_out)
-{
-    constexpr int kPer = D / 32; // 4 (D=128) or 2 (D=64) consecutive floats per lane
-    const int lane = threadIdx.x & 31;
-    float mx = -CUDART_INF_F;
-    for (int s = lane; s < n; s += 32)
-        mx = fmaxf(mx, lse[(int64_t)s * lse_stride]);
-#pragma unroll
-    for (int o2 = 16; o2; o2 >>= 1)
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
-    float acc[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i)
-        acc[i] = 0.f;
-    float z = 0.f;
-    if (mx != -CUDART_INF_F) {
-        for (int s0 = 0; s0 < n; s0 += 32) {
-            const int s = s0 + lane;
-            const float w = s < n ? __expf(lse[(int64_t)s * lse_stride] - mx) : 0.f;
-            z += w;
-            const int cnt = min(32, n - s0);
-            for (int k = 0; k < cnt; ++k) {
-                const float wk = __shfl_sync(0xffffffffu, w, k);
-                const float *src = o + (int64_t)(s0 + k) * o_stride + lane * kPer;
-                if constexpr (kPer == 4) {
-                    const float4 v = *reinterpret_cast<const float4 *>(src);
-                    acc[0] += wk * v.x;
-                    acc[1] += wk * v.y;
-                    acc[2] += wk * v.z;
-                    acc[3] += wk * v.w;
-                } else {
-                    const float2 v = *reinterpret_cast<const float2 *>(src);
-                    acc[0] += wk * v.x;
-                    acc[1] += wk * v.y;
-                }
-            }
-        }
-#pragma unroll
-        for (int o2 = 16; o2; o2 >>= 1)
-            z += __shfl_xor_sync(0xffffffffu, z, o2);
-    }
-    const float inv = z > 0.f ? 1.f / z : 0.f;
-    __nv_bfloat16 *dst = out + lane * kPer;
-    if constexpr (kPer == 4) {
-        __nv_bfloat162 a = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-        __nv_bfloat162 b = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
-        uint2 v;
-        v.x = *reinterpret_cast<uint32_t *>(&a);
-        v.y = *reinterpret_cast<uint32_t *>(&b);
-        *reinterpret_cast<uint2 *>(dst) = v;
-    } else {
-        *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-    }
-    if (lse_out && lane == 0)
-        *lse_out = z > 0.f ? mx + logf(z) : -CUDART_INF_F;
-}
-
-// Split-KV reduce of the decode requests that were split (one CTA each).
-template <int D>
-__global__ void __launch_bounds__(256) reduce_kernel(const AttnParams p)
-{
-    const int b = blockIdx.x;
-    if (b >= (int)p.hdr->n_reduce)
-        return;
-    const int r = p.red_list[b];
-    const int qs = p.qsl[r];
-    const int q_len = p.qsl[r + 1] - qs;
-    const int L = p.seq_lens[r];
-    const int n = (L + p.split_tokens - 1) / p.split_tokens;
-    const int warps = blockDim.x >> 5;
-    for (int pair = threadIdx.x >> 5; pair < q_len * p.Hq; pair += warps) {
-        const int i = pair / p.Hq, hq = pair - i * p.Hq;
-        const int64_t idx = (((int64_t)r * p.QD + i) * p.Hq + hq) * p.max_splits;
-        const int64_t orow = (int64_t)(qs + i) * p.Hq + hq;
-        merge_one<D>(p.part_o + idx * D, D, p.part_lse + idx, 1, n, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
-    }
-}
-
 template <int D>
 __global__ void __launch_bounds__(256) merge_states_kernel(const float *__restrict__ part_out,
                                                            const float *__restrict__ part_lse,
@@ -356,15 +276,6 @@ cudaError_t launch_plan(const AttnParams &p, cudaStream_t s)
         n_buckets = 12 * 1024;
     const int smem = n_buckets * (int)sizeof(int);
     plan_kernel<<<1, 1024, smem, s>>>(p, n_buckets);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_reduce(const AttnParams &p, cudaStream_t s)
-{
-    if (p.D == 128)
-        reduce_kernel<128><<<p.num_seqs, 256, 0, s>>>(p);
-    else
-        reduce_kernel<64><<<p.num_seqs, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
