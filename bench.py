@@ -2,8 +2,8 @@
 """Benchmark of the paged-attention hot path on B200.
 
 One step = one pass of the whole hot path over one batch: pa_kv_write of the
-step's new K/V rows, then pa_attention_mixed (plan, decode, split-KV reduce,
-prefill as the batch needs).  The headline workload is the Llama-3-8B-shaped
+step's new K/V rows, then pa_attention_mixed (plan, decode with its split-KV
+merge, prefill as the batch needs).  The headline workload is the Llama-3-8B-shaped
 decode batch (256 requests, context U[512, 4096], 32 q / 8 kv heads, head_dim
 128, 70k-block pool); the metric is KV bytes the attention must read per
 second (sum over requests of seq_len * Hkv * D * 2 tensors * 2 bytes, exact
@@ -193,9 +193,8 @@ class Step:
         G = lay.num_q_heads // lay.num_kv_heads
         NT = 1 if G <= 8 else (2 if G <= 16 else 0)
         cap = 8 * NT
-        max_splits = math.ceil(max(lay.max_seq_len, 1) / 1024) if NT else 0
-        self.launches_per_step = 2 + (1 if NT else 0) + (1 if NT and max_splits > 1 else 0) + \
-            (1 if lay.max_query_len * G > cap else 0)
+        # pa_kv_write, plan, decode (split merge inside), prefill when the batch has prefill work
+        self.launches_per_step = 2 + (1 if NT else 0) + (1 if lay.max_query_len * G > cap else 0)
         self.kv_bytes = lay.kv_bytes()
         q = lay.q_lens.astype(np.int64)
         c = lay.ctx_lens.astype(np.int64)
@@ -417,7 +416,7 @@ def _follow_on(st: Step, steps: int, warmup: int, peaks: dict):
                                            decode_max_query_len=dq)
     ms_dec = _time_region(spec(4, ws_dec), steps, warmup, 1) / steps
     ms_pf = _time_region(spec(0, ws_pf), steps, warmup, 1) / steps
-    launches += 7 * steps  # plan+decode+reduce; plan+decode+reduce (no work)+prefill
+    launches += 5 * steps  # plan + decode; plan + decode (no work) + prefill
     kvb = sl.kv_bytes()
     res["spec_verify_k3"] = {"value": kvb / (ms_dec * 1e-3) / 1e9, "unit": "GB/s",
                              "frac": kvb / (ms_dec * 1e-3) / 1e9 / hbm, "ms_per_launch": ms_dec,
@@ -603,13 +602,13 @@ def main():
     clocks = sampler.stop(*win)
     value, ms_step = whole_job_value(st.kv_bytes, ms_total / args.steps, ws)
 
-    # dominant kernel roofline: the attention launches (plan + decode + reduce), events on their stream
+    # dominant kernel roofline: the attention launches (plan + decode with its split merge), events on their stream
     att_ms = _attention_only_ms(st, max(20, min(args.steps, 200)))
     achieved = st.kv_bytes / (att_ms * 1e-3) / 1e9
     traffic, _ = _traffic("decode_llama3_8b_decode", ["decode.cu", "ptx.cuh", "pa_internal.cuh"])
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "pa_attention_mixed (plan + decode_kernel + reduce_kernel)",
+                "kernel": "pa_attention_mixed (plan_kernel + decode_kernel with its split merge)",
                 "algorithmic_bytes_per_launch": st.kv_bytes, "ms_per_launch": att_ms,
                 "peak_source": f"{peaks['source']} hbm_gbs (burst copy)"}
 
