@@ -458,6 +458,35 @@ def _follow_on(st: Step, steps: int, warmup: int, peaks: dict):
     return res, launches
 
 
+def _other_workloads(steps: int, warmup: int, peaks: dict):
+    """The long-context decode batch (split-KV with the in-kernel merge) and the prefix-sharing batch
+    (128 requests whose first 128 blocks are the same physical blocks): attention call only, CUDA events.
+    Prefix sharing reports the logical KV bytes the requests attend over and the unique bytes HBM must
+    deliver (the shared blocks are read once from HBM, then from L2)."""
+    import torch
+    res = {}
+    for name in ("long_context_decode", "prefix_sharing"):
+        st = Step(name)
+        st.kv_write()
+        ms = _time_region(st.attention, steps, warmup, 1) / steps
+        lay = st.lay
+        logical = lay.kv_bytes()
+        d = {"ms_per_launch": ms, "value": logical / (ms * 1e-3) / 1e9, "unit": "GB/s",
+             "frac": logical / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "workload": lay.describe()}
+        if name == "prefix_sharing":
+            # unique tokens: the shared 2048-token prefix once plus every private suffix
+            shared = 2048
+            uniq_tokens = shared + int((lay.seq_lens - shared).sum())
+            unique = uniq_tokens * lay.num_kv_heads * lay.head_dim * 2 * 2
+            d.update({"value_unique": unique / (ms * 1e-3) / 1e9,
+                      "frac_unique": unique / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                      "unique_kv_bytes": unique, "logical_kv_bytes": logical})
+        res[name] = d
+        del st
+        torch.cuda.empty_cache()
+    return res, 2 * 2 * steps  # plan + decode per call, two workloads
+
+
 def _prefix_hash_rate():
     """Host-side prefix caching on the prefix-sharing workload's shape (128 requests, 2048 shared prompt
     tokens plus private suffixes, synthetic token ids): chained block hashing of every request and the
@@ -662,6 +691,8 @@ def main():
     if not args.no_extras and rank == 0:
         line["follow_on"], n_l = _follow_on(st, max(10, min(args.steps, 50)), args.warmup, peaks)
         line["follow_on"]["prefix_hash"] = _prefix_hash_rate()
+        line["other_workloads"], n_o = _other_workloads(max(10, min(args.steps, 30)), args.warmup, peaks)
+        line["gpu_launches"] += n_o
         line["gpu_launches"] += n_l
     if not args.no_extras:
         del st
