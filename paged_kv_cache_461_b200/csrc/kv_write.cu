@@ -100,7 +100,7 @@ __global__ void gather_kernel(const uint16_t *__restrict__ cache, int64_t num_bl
 
 // Whole-block copies between the caches and a staging buffer [num_ids][2][bv] of 16-byte
 // vectors (bv vectors per block).  One unit = (entry i, cache kv) = staging row 2i+kv; CTAs
-// stride over units and each CTA's threads over the unit's vectors, four in flight per
+// stride over units and each CTA's threads over the unit's vectors, eight in flight per
 // thread.  PACK: cache -> staging (an id outside the pool gives zeros); otherwise
 // staging -> cache (an id outside the pool is skipped).
 template <bool PACK>
@@ -109,9 +109,13 @@ __global__ void __launch_bounds__(256) kv_block_copy_kernel(uint4 *__restrict__ 
                                                             const int32_t *__restrict__ ids, int64_t n_units,
                                                             uint4 *__restrict__ staging)
 {
-    constexpr int kU = 4;
+    constexpr int kU = 8;
+    // the next unit's block id is loaded while this unit is copied
+    int64_t bid_next = blockIdx.x < n_units ? ids[blockIdx.x >> 1] : 0;
     for (int64_t unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
-        const int64_t bid = ids[unit >> 1];
+        const int64_t bid = bid_next;
+        const int64_t nu = unit + gridDim.x;
+        bid_next = nu < n_units ? ids[nu >> 1] : 0;
         const bool ok = bid >= 0 && bid < num_blocks;
         if (!PACK && !ok)
             continue;

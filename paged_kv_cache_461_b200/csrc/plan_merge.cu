@@ -172,10 +172,14 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
     };
     // pass 1: decode units and reduce list in request order; histogram of prefill pair costs
     int carry_dec = 0, carry_pf = 0, carry_red = 0;
+    int kept_pf = 0, kept_ctx = 0, kept_q = 0; // this thread's request when one pass covers them all
     for (int base = 0; base < p.num_seqs; base += blockDim.x) {
         const int r = base + threadIdx.x;
         int n_dec, n_pf, red, ctx, q_len;
         classify(r, n_dec, n_pf, red, ctx, q_len);
+        kept_pf = n_pf;
+        kept_ctx = ctx;
+        kept_q = q_len;
         for (int k = 0; k < n_pf; ++k)
             atomicAdd(&hist[min(pair_cost(ctx, q_len, k, tq), n_buckets - 1)], 1);
         if (n_dec)
@@ -194,26 +198,30 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
         carry_red += tr;
     }
     __syncthreads();
-    // bucket start offsets, most expensive bucket first
-    int carry = 0;
-    for (int base = 0; base < n_buckets; base += blockDim.x) {
-        const int b = n_buckets - 1 - (base + (int)threadIdx.x); // descending cost
-        const int cnt = b >= 0 ? hist[b] : 0;
-        int e0, e1, e2, t0, t1, t2;
-        cta_excl_scan3(cnt, 0, 0, e0, e1, e2, t0, t1, t2);
-        if (b >= 0)
-            hist[b] = carry + e0;
-        carry += t0;
-        __syncthreads();
-    }
-    // pass 2: scatter the prefill pairs into their cost buckets
-    for (int base = 0; base < p.num_seqs; base += blockDim.x) {
-        const int r = base + threadIdx.x;
-        int n_dec, n_pf, red, ctx, q_len;
-        classify(r, n_dec, n_pf, red, ctx, q_len);
-        for (int k = 0; k < n_pf; ++k) {
-            const int pos = atomicAdd(&hist[min(pair_cost(ctx, q_len, k, tq), n_buckets - 1)], 1);
-            p.pf_tiles[pos] = make_int2(r, k);
+    if (carry_pf > 0) { // a step without prefill work skips the sort
+        // bucket start offsets, most expensive bucket first
+        int carry = 0;
+        for (int base = 0; base < n_buckets; base += blockDim.x) {
+            const int b = n_buckets - 1 - (base + (int)threadIdx.x); // descending cost
+            const int cnt = b >= 0 ? hist[b] : 0;
+            int e0, e1, e2, t0, t1, t2;
+            cta_excl_scan3(cnt, 0, 0, e0, e1, e2, t0, t1, t2);
+            if (b >= 0)
+                hist[b] = carry + e0;
+            carry += t0;
+            __syncthreads();
+        }
+        // pass 2: scatter the prefill pairs into their cost buckets (requests re-read only when
+        // there are more of them than threads)
+        for (int base = 0; base < p.num_seqs; base += blockDim.x) {
+            const int r = base + threadIdx.x;
+            int n_dec, n_pf = kept_pf, red, ctx = kept_ctx, q_len = kept_q;
+            if (p.num_seqs > (int)blockDim.x)
+                classify(r, n_dec, n_pf, red, ctx, q_len);
+            for (int k = 0; k < n_pf; ++k) {
+                const int pos = atomicAdd(&hist[min(pair_cost(ctx, q_len, k, tq), n_buckets - 1)], 1);
+                p.pf_tiles[pos] = make_int2(r, k);
+            }
         }
     }
     // block sums of the two estimates (warp shuffles, then one warp over the warp partials)
