@@ -154,7 +154,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
         : "r"(taddr));
 }
 
-// same as tmem_ld32, into r[0..31] of a larger register array (constant indices only)
+// 32 lanes x 32 consecutive 32-bit columns into r[0..31] of a register array (constant indices only):
+// thread i of the warp gets lane (base + i), columns col .. col + 31
 __device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t *r)
 {
     asm volatile(
