@@ -586,6 +586,7 @@ def reference_arm(args, ws, rank):
 def profile_case(kind: str, launches: int):
     """A reduced copy of a workload for ncu (same shapes, fewer requests, pool sized to fit):
     decode: the first 64 requests of the Llama-3-8B-shaped decode batch (~0.6 GB of KV, above L2);
+    spec: the same 64 requests verifying 3 drafted tokens each (q_len 4, decode_max_query_len 4);
     prefill: the prefill chunks of the mixed 8192-token step alone.
     Runs 1 warm-up launch of pa_attention_mixed and then `launches` more."""
     import torch
@@ -593,13 +594,14 @@ def profile_case(kind: str, launches: int):
     from paged_kv_cache_461_b200 import api, build
     from paged_kv_cache_461_b200 import workloads as W
     build.build()
-    full = W.workload_layout(HEADLINE if kind == "decode" else MIXED)
-    if kind == "decode":
+    full = W.workload_layout(MIXED if kind == "prefill" else HEADLINE)
+    if kind in ("decode", "spec"):
         idx = np.arange(64)
     else:
         G = full.num_q_heads // full.num_kv_heads
         idx = np.nonzero(full.q_lens * G > 8)[0]
-    lay = W.build_layout(f"{full.name}_{kind}_case", full.ctx_lens[idx], full.q_lens[idx],
+    q_lens = np.full(len(idx), 4, np.int32) if kind == "spec" else full.q_lens[idx]
+    lay = W.build_layout(f"{full.name}_{kind}_case", full.ctx_lens[idx], q_lens,
                          num_q_heads=full.num_q_heads, num_kv_heads=full.num_kv_heads, head_dim=full.head_dim,
                          seed=full.seed)
     v = W.make_values_torch(lay, "cuda")
@@ -608,7 +610,8 @@ def profile_case(kind: str, launches: int):
     bt = torch.from_numpy(lay.block_table).cuda()
     slots = torch.from_numpy(lay.slot_mapping).cuda()
     api.kv_write(v.k_new, v.v_new, slots, v.k_cache, v.v_cache)
-    dq = -1 if kind == "prefill" else 0   # the prefill chunks as a prefill-only batch, as bench.py times them
+    # the prefill chunks as a prefill-only batch, as bench.py times them; verify shapes on the decode kernel
+    dq = {"prefill": -1, "spec": 4}.get(kind, 0)
     ws = api.alloc_workspace(lay.num_seqs, lay.num_tokens, lay.num_q_heads, v.k_cache, lay.max_seq_len,
                              decode_max_query_len=dq)
     out = torch.empty_like(v.q)
@@ -631,7 +634,7 @@ def main():
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="headline only (no mixed step, e2e, prefill)")
-    ap.add_argument("--profile-case", choices=["decode", "prefill"],
+    ap.add_argument("--profile-case", choices=["decode", "spec", "prefill"],
                     help="run a small case of one kernel for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:

@@ -446,16 +446,20 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
     if (n_splits == 1)
         return;
     // Split request: the last of its split CTAs for this kv head merges all the splits' states.
-    // Release: every thread's partial stores are made visible before the arrival is counted.
-    __threadfence();
-    __syncthreads();
+    // Release: the CTA barrier orders every thread's partial stores before thread 0's fence and
+    // arrival (fences are cumulative); acquire: thread 0 fences after seeing the last arrival and
+    // the barrier orders the other threads' reads (past L1) after it.
     __shared__ int s_last;
-    if (threadIdx.x == 0)
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
         s_last = atomicAdd(&p.split_arrivals[(int64_t)r * p.Hkv + h], 1u) == (unsigned)(n_splits - 1);
+        if (s_last)
+            __threadfence();
+    }
     __syncthreads();
     if (!s_last)
         return;
-    __threadfence(); // acquire: the other splits' states, read below past L1
     for (int rr = warp; rr < rows; rr += kDecWarps) {
         const int t = qs + rr / p.G;
         const int hq = h * p.G + rr % p.G;
