@@ -11,9 +11,10 @@
 //
 // Data path per CTA (4 warps):
 //   * each warp owns every 4th 16-token block of the split and a private ring
-//     of kStages stages; lane 0 fetches one (block, kv head) K tile and V tile
-//     with 2-D TMA loads (128-byte swizzled, 2 KiB per 64-column half) that
-//     complete on the stage's mbarrier, kStages blocks ahead of use;
+//     of 3 stages (2 when 16 rows are packed, so 3 CTAs fit per SM); lane 0
+//     fetches one (block, kv head) K tile and V tile with TMA loads (128-byte
+//     swizzled, 2 KiB per 64-column half) that complete on the stage's
+//     mbarrier, one ring ahead of use;
 //   * S^T = K Q^T on mma.sync m16n8k16 (keys are the M=16 rows: one paged
 //     block per MMA), bf16 in, fp32 accumulate; Q^T fragments stay in
 //     registers for the whole split;
@@ -39,15 +40,17 @@ namespace pa {
 namespace {
 
 constexpr int kDecWarps = 4;
-constexpr int kDecStages = 3;
 
-template <int D>
+// Ring depth per warp: 3 blocks for 8 packed rows (2 CTAs per SM), 2 for 16 rows, where
+// each block takes twice the work and 3 CTAs per SM (12 warps) hide more of it.
+template <int D, int NT>
 struct DecCfg {
+    static constexpr int kStages = NT == 1 ? 3 : 2;
     static constexpr int kHalves = D / 64;
     static constexpr int kBox = 16 * 64 * 2;           // one TMA box: 16 rows x 64 bf16
     static constexpr int kTile = kHalves * kBox;       // one (block, kv head) of K or V
     static constexpr int kStage = 2 * kTile;           // K + V
-    static constexpr int kData = kDecWarps * kDecStages * kStage;
+    static constexpr int kData = kDecWarps * kStages * kStage;
     static constexpr int kSmem = kData + 64 * 8 + 1024; // + barriers + alignment slack
 };
 
@@ -63,7 +66,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
                                                                 const __grid_constant__ CUtensorMap tm_v,
                                                                 const AttnParams p)
 {
-    using Cfg = DecCfg<D>;
+    using Cfg = DecCfg<D, NT>;
+    constexpr int kDecStages = Cfg::kStages;
     constexpr int kKS = D / 16; // k-steps of S^T over the head dim
     constexpr int kMT = D / 16; // m-tiles of O^T over the head dim
     constexpr int kRows = 8 * NT;
@@ -474,7 +478,7 @@ template <int D, int NT>
 cudaError_t launch_decode_t(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int64_t grid_units,
                             cudaStream_t s)
 {
-    constexpr int smem = DecCfg<D>::kSmem;
+    constexpr int smem = DecCfg<D, NT>::kSmem;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
