@@ -241,3 +241,36 @@ def test_step_replays_from_a_cuda_graph_bit_identically(kind):
     torch.cuda.synchronize()
     assert _bits_equal(out_g, out_e) and torch.equal(lse_g, lse_e)
     assert api.read_device_status(st.workspace) == 0
+
+
+@pytest.mark.parametrize("mode", ["fused_decode", "prefill_only"])
+def test_other_entry_points_replay_from_a_cuda_graph(mode):
+    rng = np.random.default_rng(41)
+    if mode == "fused_decode":
+        ctx, q = list(rng.integers(0, 2500, size=30)), [1] * 30
+    else:
+        ctx, q = [0, 300, 1200], [400, 129, 77]
+    lay = _layout("graph2", ctx, q, 32, 8, 128, seed=19)
+    vals = W.make_values_numpy(lay, sentinel="pattern")
+    st = DevStep(lay, vals)
+    if mode == "fused_decode":
+        out_e, lse_e = st.write_and_attend_fused()
+        call = lambda o, l: api.attention_decode_fused(st.q, st.k_new, st.v_new, st.k_cache, st.v_cache, st.qsl,
+                                                       st.seq_lens, st.bt, lay.max_query_len, lay.max_seq_len,
+                                                       out=o, lse=l, workspace=st.workspace)
+    else:
+        st.write()
+        out_e, lse_e = st.attend(decode_max_query_len=-1)
+        call = lambda o, l: api.attention_mixed(st.q, st.k_cache, st.v_cache, st.qsl, st.seq_lens, st.bt,
+                                                lay.max_query_len, lay.max_seq_len, out=o, lse=l,
+                                                workspace=st.workspace, decode_max_query_len=-1)
+    torch.cuda.synchronize()
+    out_g = torch.full_like(out_e, float("nan"))
+    lse_g = torch.full_like(lse_e, float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(out_g, lse_g)
+    g.replay()
+    torch.cuda.synchronize()
+    assert _bits_equal(out_g, out_e) and torch.equal(lse_g, lse_e)
+    assert api.read_device_status(st.workspace) == 0
