@@ -1,5 +1,5 @@
 // plan_merge.cu -- device-side work decomposition of a mixed step, and the
-// split-KV reduce (merge of attention states over disjoint key ranges).
+// stand-alone merge of attention states over disjoint key ranges.
 //
 // Plan: one CTA reads query_start_loc / seq_lens, classifies each request as
 // decode (q_len * G small enough for the warp-MMA decode kernel) or prefill
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
             n_pf = (q_len * p.G + kPrefillRowsPerCta - 1) / kPrefillRowsPerCta;
         }
     };
-    // pass 1: decode units and reduce list in request order; histogram of prefill pair costs
+    // pass 1: decode units in request order, split-arrival counters zeroed; histogram of prefill pair costs
     int carry_dec = 0, carry_pf = 0, carry_red = 0;
     int kept_pf = 0, kept_ctx = 0, kept_q = 0; // this thread's request when one pass covers them all
     for (int base = 0; base < p.num_seqs; base += blockDim.x) {
