@@ -543,16 +543,47 @@ def cpu_oracle_run(name: str, target_s: float = 15.0, seed=None):
         kc, vc = oracle.kv_write(vals.k_new, vals.v_new, sub.slot_mapping, vals.k_cache, vals.v_cache)
         t0 = time.perf_counter()
         oracle.attention_for(sub, kc, vc, vals.q)
-        return sub, time.perf_counter() - t0
+        return sub, (kc, vc, vals.q), time.perf_counter() - t0
 
-    sub, dt = run(min(8, full))
+    sub, arrs, dt = run(min(8, full))
     n = int(min(full, max(sub.num_seqs, sub.num_seqs * target_s / max(dt, 1e-3))))
     if n > sub.num_seqs:
-        sub, dt = run(n)
+        sub, arrs, dt = run(n)
     cores = oracle.num_cores()
+
+    # the same oracle on one thread, over the queries of the first m requests (about 3 s)
+    def kv_bytes_of(m):
+        return int(sub.seq_lens[:m].astype(np.int64).sum()) * sub.num_kv_heads * sub.head_dim * 2 * 2
+
+    def run1(m):
+        toks = np.arange(int(sub.query_start_loc[m]), dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.attention_for(sub, *arrs, token_list=toks, nthreads=1)
+        return time.perf_counter() - t0
+
+    m = min(2, sub.num_seqs)
+    dt1 = run1(m)
+    m2 = int(min(sub.num_seqs, max(m, m * 3.0 / max(dt1, 1e-3))))
+    if m2 > m:
+        m, dt1 = m2, run1(m2)
     return {"value": sub.kv_bytes() / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"first {sub.num_seqs} of the {full} requests of {name} "
-                      f"({sub.kv_bytes() / 1e9:.3f} GB of KV, {dt:.2f} s, fp64, {cores} threads)"}
+                      f"({sub.kv_bytes() / 1e9:.3f} GB of KV, {dt:.2f} s, fp64, {cores} threads)",
+            "single_thread": {"value": kv_bytes_of(m) / dt1 / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": f"queries of the first {m} requests of {name} "
+                                        f"({kv_bytes_of(m) / 1e9:.3f} GB of KV, {dt1:.2f} s, fp64, 1 thread)"},
+            "cpu_model": _cpu_model()}
+
+
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def reference_arm(args, ws, rank):
