@@ -296,6 +296,26 @@ def test_stress_inputs(kind):
     assert_parity(out, ref, lse, ref_lse, what=kind)
 
 
+@pytest.mark.parametrize("growth", ["jump", "ramp"])
+def test_prefill_row_max_growing_in_later_key_steps(growth):
+    # This step's keys at later positions score far above the first 128-key step's row max
+    # (x16 past position 300: ~20 in the exp2 domain above it), or climb step after step
+    # (x(1 + pos/64)), so the softmax must move its reference max past the 2^8 slack in later
+    # steps, recompute P and rescale O -- in every warp ("jump") or in a mix of warps ("ramp").
+    lay = _layout("grow", [0, 200], [600, 300], 32, 8, 128, seed=31)
+    vals = W.make_values_numpy(lay)
+    k = W.bf16_bits_to_f32(vals.k_new)
+    qsl = lay.query_start_loc
+    for r in range(lay.num_seqs):
+        pos = lay.ctx_lens[r] + np.arange(qsl[r + 1] - qsl[r])
+        f = np.where(pos >= 300, 16.0, 1.0) if growth == "jump" else 1.0 + pos / 64.0
+        k[qsl[r]:qsl[r + 1]] *= f[:, None, None].astype(np.float32)
+    vals.k_new = W.f32_to_bf16_bits(k)
+    st, out, lse, ref, ref_lse = _run(lay, vals=vals)
+    assert_parity(out, ref, lse, ref_lse, what=f"prefill, row max growing ({growth})")
+    assert api.read_device_status(st.workspace) == 0
+
+
 def test_empty_requests_and_padding_rows_are_left_alone():
     lay = _layout("e", [10, 40, 0, 300], [0, 1, 0, 70], 32, 8, 128, seed=14)
     vals = W.make_values_numpy(lay)
