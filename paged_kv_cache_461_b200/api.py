@@ -145,9 +145,65 @@ def _opts(kv_split_tokens: int, decode_max_query_len: int = 0) -> Optional[AttnO
     return o
 
 
-def _need(t: torch.Tensor, dtype, name: str):
-    if t.dtype != dtype or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA {dtype} tensor (got {t.dtype} on {t.device})")
+def _need(t: torch.Tensor, dtype, name: str, shape=None, dense: bool = False, device=None):
+    """The library sees raw pointers only, so every tensor is checked here: dtype, then CUDA
+    (and the same device as the call's other tensors), then contiguity and shape where the C
+    layout has no strides."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor (got {type(t).__name__})")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (got {t.device})")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call's other tensors on {device}")
+    if dense and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+
+
+def _need_caches(k_cache: torch.Tensor, v_cache: torch.Tensor, device=None):
+    _need(k_cache, torch.bfloat16, "k_cache", dense=True, device=device)
+    if k_cache.dim() != 4:
+        raise ValueError(f"k_cache must be 4-D (got {tuple(k_cache.shape)})")
+    _need(v_cache, torch.bfloat16, "v_cache", shape=k_cache.shape, dense=True, device=k_cache.device)
+
+
+def _need_meta(query_start_loc: torch.Tensor, seq_lens: torch.Tensor, block_table: torch.Tensor, device):
+    """query_start_loc int32 [R+1], seq_lens int32 [R], block_table int32 [R, >= blocks] with unit column
+    stride (its row stride is passed as bt_stride)."""
+    _need(seq_lens, torch.int32, "seq_lens", dense=True, device=device)
+    if seq_lens.dim() != 1:
+        raise ValueError("seq_lens must be 1-D")
+    R = seq_lens.shape[0]
+    _need(query_start_loc, torch.int32, "query_start_loc", shape=(R + 1,), dense=True, device=device)
+    _need(block_table, torch.int32, "block_table", device=device)
+    if block_table.dim() != 2 or block_table.shape[0] != R or (block_table.numel() and block_table.stride(1) != 1):
+        raise ValueError("block_table must be int32 [num_seqs, max_blocks] with unit column stride")
+
+
+def _need_new_rows(k_new: torch.Tensor, v_new: torch.Tensor, d: CacheDesc, device) -> int:
+    """k_new/v_new [T, Hkv, D] bf16 whose rows may be strided (views into a fused QKV); returns the row stride."""
+    _need(k_new, torch.bfloat16, "k_new", device=device)
+    _need(v_new, torch.bfloat16, "v_new", shape=k_new.shape, device=device)
+    if k_new.dim() != 3 or tuple(k_new.shape[1:]) != (d.num_kv_heads, d.head_dim):
+        raise ValueError(f"k_new must be [T, {d.num_kv_heads}, {d.head_dim}] (got {tuple(k_new.shape)})")
+    T = k_new.shape[0]
+    if T and (k_new.stride(0) != v_new.stride(0) or k_new.stride(-1) != 1 or k_new.stride(-2) != k_new.shape[-1]
+              or v_new.stride(-1) != 1 or v_new.stride(-2) != v_new.shape[-1]):
+        raise ValueError("k_new and v_new need the same row stride and contiguous [Hkv, D] rows")
+    return k_new.stride(0) if T else k_new.shape[-1] * k_new.shape[-2]
+
+
+def _need_q_out(q: torch.Tensor, out: Optional[torch.Tensor], lse: Optional[torch.Tensor]):
+    _need(q, torch.bfloat16, "q", dense=True)
+    if q.dim() != 3:
+        raise ValueError(f"q must be [num_tokens, num_q_heads, head_dim] (got {tuple(q.shape)})")
+    if out is not None:
+        _need(out, torch.bfloat16, "out", shape=q.shape, dense=True, device=q.device)
+    if lse is not None:
+        _need(lse, torch.float32, "lse", shape=q.shape[:2], dense=True, device=q.device)
 
 
 # ---------------------------------------------------------------- entry points
@@ -159,21 +215,21 @@ def abi_version() -> int:
 def kv_write(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, k_cache: torch.Tensor,
              v_cache: torch.Tensor, stream=None, layout: str = "HND") -> None:
     """pa_kv_write: k_new/v_new [T, Hkv, D] (rows may be strided), slot_mapping int64 [T]."""
-    _need(k_new, torch.bfloat16, "k_new")
-    _need(slot_mapping, torch.int64, "slot_mapping")
-    T = slot_mapping.shape[0]
-    row_stride = k_new.stride(0) if T else k_new.shape[-1] * k_new.shape[-2]
-    if k_new.stride(0) != v_new.stride(0) or k_new.stride(-1) != 1 or k_new.stride(-2) != k_new.shape[-1]:
-        raise ValueError("k_new and v_new need the same row stride and contiguous [Hkv, D] rows")
+    _need_caches(k_cache, v_cache)
     d = cache_desc(k_cache, layout)
+    row_stride = _need_new_rows(k_new, v_new, d, k_cache.device)
+    T = k_new.shape[0]
+    _need(slot_mapping, torch.int64, "slot_mapping", shape=(T,), dense=True, device=k_cache.device)
     _check(lib().pa_kv_write(_ptr(k_new), _ptr(v_new), row_stride, _ptr(slot_mapping), T, _ptr(k_cache),
                              _ptr(v_cache), ctypes.byref(d), _stream(stream)), "pa_kv_write")
 
 
 def build_slot_mapping(query_start_loc: torch.Tensor, seq_lens: torch.Tensor, block_table: torch.Tensor,
                        num_tokens: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _need_meta(query_start_loc, seq_lens, block_table, query_start_loc.device)
     if out is None:
         out = torch.full((num_tokens,), -1, dtype=torch.int64, device=query_start_loc.device)
+    _need(out, torch.int64, "out", shape=(num_tokens,), dense=True, device=query_start_loc.device)
     _check(lib().pa_build_slot_mapping(_ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
                                        block_table.stride(0), seq_lens.shape[0], num_tokens, _ptr(out),
                                        _stream(stream)), "pa_build_slot_mapping")
@@ -204,7 +260,9 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
                     kv_split_tokens: int = 0, decode_max_query_len: int = 0, stream=None,
                     layout: str = "HND") -> torch.Tensor:
     """pa_attention_mixed[_ex]: q [T, Hq, D] bf16 -> out [T, Hq, D] bf16 (lse [T, Hq] fp32 if given)."""
-    _need(q, torch.bfloat16, "q")
+    _need_q_out(q, out, lse)
+    _need_caches(k_cache, v_cache, q.device)
+    _need_meta(query_start_loc, seq_lens, block_table, q.device)
     T, Hq, D = q.shape
     R = seq_lens.shape[0]
     if softmax_scale is None:
@@ -213,6 +271,7 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len, layout)
+    _need(workspace, torch.uint8, "workspace", dense=True, device=q.device)
     d = cache_desc(k_cache, layout)
     o = _opts(kv_split_tokens, decode_max_query_len)
     _check(lib().pa_attention_mixed_ex(_ptr(q), Hq, _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
@@ -231,7 +290,9 @@ def attention_mixed_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
                             kv_split_tokens: int = 0, stream=None, layout: str = "HND") -> torch.Tensor:
     """pa_attention_mixed_noalloc: like attention_mixed but with the library's built-in scratch
     (for callers that cannot allocate a workspace; calls that overlap on the GPU race on it)."""
-    _need(q, torch.bfloat16, "q")
+    _need_q_out(q, out, lse)
+    _need_caches(k_cache, v_cache, q.device)
+    _need_meta(query_start_loc, seq_lens, block_table, q.device)
     T, Hq, D = q.shape
     R = seq_lens.shape[0]
     if softmax_scale is None:
@@ -258,20 +319,22 @@ def attention_decode_fused(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Te
                            layout: str = "HND") -> torch.Tensor:
     """pa_attention_decode_fused: writes k_new/v_new [T, Hkv, D] (rows may be strided) into their
     slots and attends, in the decode kernel; every request must be decode-shaped."""
-    _need(q, torch.bfloat16, "q")
-    _need(k_new, torch.bfloat16, "k_new")
+    _need_q_out(q, out, lse)
+    _need_caches(k_cache, v_cache, q.device)
+    _need_meta(query_start_loc, seq_lens, block_table, q.device)
+    d = cache_desc(k_cache, layout)
+    row_stride = _need_new_rows(k_new, v_new, d, q.device)
     T, Hq, D = q.shape
     R = seq_lens.shape[0]
-    if k_new.stride(0) != v_new.stride(0) or k_new.stride(-1) != 1 or k_new.stride(-2) != k_new.shape[-1]:
-        raise ValueError("k_new and v_new need the same row stride and contiguous [Hkv, D] rows")
-    row_stride = k_new.stride(0) if T else k_new.shape[-1] * k_new.shape[-2]
+    if k_new.shape[0] != T:
+        raise ValueError(f"k_new has {k_new.shape[0]} rows, q has {T} tokens")
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len, layout)
-    d = cache_desc(k_cache, layout)
+    _need(workspace, torch.uint8, "workspace", dense=True, device=q.device)
     o = _opts(kv_split_tokens, decode_max_query_len)
     _check(lib().pa_attention_decode_fused(_ptr(q), Hq, _ptr(k_new), _ptr(v_new), row_stride, _ptr(k_cache),
                                            _ptr(v_cache), ctypes.byref(d), _ptr(query_start_loc), _ptr(seq_lens),
@@ -286,12 +349,14 @@ def attention_decode_fused(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Te
 def kv_pack(k_cache: torch.Tensor, v_cache: torch.Tensor, block_ids: torch.Tensor,
             staging: Optional[torch.Tensor] = None, stream=None, layout: str = "HND") -> torch.Tensor:
     """pa_kv_pack: whole blocks block_ids (int32) -> staging bf16 [n, 2, block_elems]."""
-    _need(block_ids, torch.int32, "block_ids")
+    _need_caches(k_cache, v_cache)
+    _need(block_ids, torch.int32, "block_ids", dense=True, device=k_cache.device)
     d = cache_desc(k_cache, layout)
     n = block_ids.shape[0]
     elems = d.num_kv_heads * d.block_size * d.head_dim
     if staging is None:
         staging = torch.empty((n, 2, elems), dtype=k_cache.dtype, device=k_cache.device)
+    _need(staging, torch.bfloat16, "staging", shape=(n, 2, elems), dense=True, device=k_cache.device)
     _check(lib().pa_kv_pack(_ptr(k_cache), _ptr(v_cache), ctypes.byref(d), _ptr(block_ids), n, _ptr(staging),
                             _stream(stream)), "pa_kv_pack")
     return staging
@@ -300,8 +365,12 @@ def kv_pack(k_cache: torch.Tensor, v_cache: torch.Tensor, block_ids: torch.Tenso
 def kv_unpack(staging: torch.Tensor, block_ids: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
               stream=None, layout: str = "HND") -> None:
     """pa_kv_unpack: staging bf16 [n, 2, block_elems] -> whole blocks block_ids of the caches."""
-    _need(block_ids, torch.int32, "block_ids")
+    _need_caches(k_cache, v_cache)
+    _need(block_ids, torch.int32, "block_ids", dense=True, device=k_cache.device)
     d = cache_desc(k_cache, layout)
+    n = block_ids.shape[0]
+    _need(staging, torch.bfloat16, "staging", shape=(n, 2, d.num_kv_heads * d.block_size * d.head_dim), dense=True,
+          device=k_cache.device)
     _check(lib().pa_kv_unpack(_ptr(staging), _ptr(block_ids), block_ids.shape[0], _ptr(k_cache), _ptr(v_cache),
                               ctypes.byref(d), _stream(stream)), "pa_kv_unpack")
 
@@ -310,9 +379,19 @@ def merge_attn_states(part_out: torch.Tensor, part_lse: torch.Tensor, parts_per_
                       out: Optional[torch.Tensor] = None, lse_out: Optional[torch.Tensor] = None,
                       stream=None) -> torch.Tensor:
     """pa_merge_attn_states: part_out fp32 [N, H, S, D], part_lse fp32 [N, H, S] -> bf16 [N, H, D]."""
+    _need(part_out, torch.float32, "part_out", dense=True)
+    if part_out.dim() != 4:
+        raise ValueError(f"part_out must be [N, H, S, D] (got {tuple(part_out.shape)})")
     N, H, S, D = part_out.shape
+    dev = part_out.device
+    _need(part_lse, torch.float32, "part_lse", shape=(N, H, S), dense=True, device=dev)
+    if parts_per_row is not None:
+        _need(parts_per_row, torch.int32, "parts_per_row", shape=(N,), dense=True, device=dev)
     if out is None:
-        out = torch.empty((N, H, D), dtype=torch.bfloat16, device=part_out.device)
+        out = torch.empty((N, H, D), dtype=torch.bfloat16, device=dev)
+    _need(out, torch.bfloat16, "out", shape=(N, H, D), dense=True, device=dev)
+    if lse_out is not None:
+        _need(lse_out, torch.float32, "lse_out", shape=(N, H), dense=True, device=dev)
     _check(lib().pa_merge_attn_states(_ptr(part_out), _ptr(part_lse), _ptr(parts_per_row), N, H, S, D, _ptr(out),
                                       _ptr(lse_out), _stream(stream)), "pa_merge_attn_states")
     return out
@@ -320,7 +399,11 @@ def merge_attn_states(part_out: torch.Tensor, part_lse: torch.Tensor, parts_per_
 
 def debug_gather_kv(cache: torch.Tensor, bt_row: torch.Tensor, seq_len: int, stream=None,
                     layout: str = "HND") -> torch.Tensor:
+    _need(cache, torch.bfloat16, "cache", dense=True)
+    _need(bt_row, torch.int32, "bt_row", dense=True, device=cache.device)
     d = cache_desc(cache, layout)
+    if bt_row.numel() < (seq_len + d.block_size - 1) // d.block_size:
+        raise ValueError("bt_row holds fewer block ids than seq_len needs")
     out = torch.empty((seq_len, d.num_kv_heads, d.head_dim), dtype=cache.dtype, device=cache.device)
     _check(lib().pa_debug_gather_kv(_ptr(cache), ctypes.byref(d), _ptr(bt_row), seq_len, _ptr(out),
                                     _stream(stream)), "pa_debug_gather_kv")
@@ -372,7 +455,8 @@ class PrefixCache:
         import numpy as np
         h = np.ascontiguousarray(hashes, dtype=np.uint8).reshape(-1, 32)
         b = np.ascontiguousarray(block_ids, dtype=np.int32)
-        assert len(h) == len(b)
+        if len(h) != len(b):
+            raise ValueError(f"{len(h)} hashes but {len(b)} block ids")
         _check(lib().pa_prefix_cache_insert(self._h, h.ctypes.data, b.ctypes.data, len(b)), "pa_prefix_cache_insert")
 
     def remove_block(self, block_id: int) -> None:

@@ -201,3 +201,48 @@ def test_fused_decode_host_validation(L):
     assert _fused(L, stride=1028) == 2                   # not a multiple of 8 elements
     assert _fused(L, kn=FAKE + (1 << 33) + 2) == 2       # k_new not 16-byte aligned
     assert _fused(L, hq=8 * 3) == 2
+
+
+def test_binding_rejects_host_tensors_before_the_library(L):
+    # every GPU entry point of the binding refuses host (CPU) tensors with a TypeError: there is
+    # no CPU fallback, and nothing reaches the library
+    import torch
+    bf = torch.bfloat16
+    q = torch.zeros(4, 2, 64, dtype=bf)
+    kc = torch.zeros(8, 2, 16, 64, dtype=bf)
+    vc = torch.zeros_like(kc)
+    kn = torch.zeros(4, 2, 64, dtype=bf)
+    qsl = torch.arange(5, dtype=torch.int32)
+    sl = torch.full((4,), 5, dtype=torch.int32)
+    bt = torch.zeros(4, 2, dtype=torch.int32)
+    slots = torch.zeros(4, dtype=torch.int64)
+    ids = torch.zeros(3, dtype=torch.int32)
+    calls = [
+        lambda: api.kv_write(kn, kn, slots, kc, vc),
+        lambda: api.build_slot_mapping(qsl, sl, bt, 4),
+        lambda: api.attention_mixed(q, kc, vc, qsl, sl, bt, 1, 5),
+        lambda: api.attention_mixed_noalloc(q, kc, vc, qsl, sl, bt, 1, 5),
+        lambda: api.attention_decode_fused(q, kn, kn, kc, vc, qsl, sl, bt, 1, 5),
+        lambda: api.kv_pack(kc, vc, ids),
+        lambda: api.kv_unpack(torch.zeros(3, 2, 2048, dtype=bf), ids, kc, vc),
+        lambda: api.merge_attn_states(torch.zeros(2, 2, 3, 64), torch.zeros(2, 2, 3)),
+        lambda: api.debug_gather_kv(kc, bt[0], 5),
+    ]
+    for call in calls:
+        with pytest.raises(TypeError, match="CUDA"):
+            call()
+
+
+def test_binding_checks_dtype_before_device(L):
+    import torch
+    with pytest.raises(TypeError, match="int32"):
+        api._need(torch.zeros(3, dtype=torch.int64), torch.int32, "seq_lens")
+    with pytest.raises(TypeError, match="bfloat16"):
+        api._need(torch.zeros(3, 2, 64), torch.bfloat16, "q")
+    with pytest.raises(TypeError, match="torch tensor"):
+        api._need([1, 2, 3], torch.int32, "seq_lens")
+    c = api.PrefixCache()
+    h = api.prefix_block_hashes(list(range(32)))
+    with pytest.raises(ValueError, match="block ids"):
+        c.insert(h, [1])
+    c.close()

@@ -274,3 +274,44 @@ def test_other_entry_points_replay_from_a_cuda_graph(mode):
     torch.cuda.synchronize()
     assert _bits_equal(out_g, out_e) and torch.equal(lse_g, lse_e)
     assert api.read_device_status(st.workspace) == 0
+
+
+# ----------------------------------------------------------------------------- binding argument checks
+
+def test_binding_rejects_malformed_tensors_before_launching():
+    # The C ABI sees pointers only; the binding checks dtype, device, contiguity and shapes first.
+    lay = _layout("args", [17, 40, 3], [1, 1, 1], 8, 2, 128, seed=41)
+    st = DevStep(lay, W.make_values_numpy(lay))
+    st.write()
+    T, Hq = lay.num_tokens, lay.num_q_heads
+
+    def attend(**kw):
+        a = dict(q=st.q, k_cache=st.k_cache, v_cache=st.v_cache, query_start_loc=st.qsl, seq_lens=st.seq_lens,
+                 block_table=st.bt, max_query_len=lay.max_query_len, max_seq_len=lay.max_seq_len)
+        a.update(kw)
+        return api.attention_mixed(**a)
+
+    with pytest.raises(TypeError, match="int32"):
+        attend(seq_lens=st.seq_lens.long())
+    with pytest.raises(TypeError, match="CUDA"):
+        attend(query_start_loc=st.qsl.cpu())
+    with pytest.raises(ValueError, match="contiguous"):
+        attend(q=st.q.transpose(0, 1).contiguous().transpose(0, 1))
+    with pytest.raises(ValueError, match="shape"):
+        attend(lse=torch.empty(T, Hq + 1, device="cuda"))
+    with pytest.raises(ValueError, match="block_table"):
+        attend(block_table=st.bt[:-1])
+    with pytest.raises(ValueError, match="v_cache"):
+        attend(v_cache=st.v_cache[:-1])
+    with pytest.raises(ValueError, match="slot_mapping"):
+        api.kv_write(st.k_new, st.v_new, st.slots[:-1], st.k_cache, st.v_cache)
+    with pytest.raises(TypeError, match="float32"):
+        api.merge_attn_states(torch.zeros(2, 2, 3, 128, device="cuda"), torch.zeros(2, 2, 3, device="cuda"),
+                              lse_out=torch.zeros(2, 2, device="cuda", dtype=torch.float64))
+    # a block table wider than needed, as a column slice of a wider one, is still accepted
+    wide = torch.full((lay.num_seqs, st.bt.shape[1] + 5), -1, dtype=torch.int32, device="cuda")
+    wide[:, :st.bt.shape[1]] = st.bt
+    got = attend(block_table=wide[:, :st.bt.shape[1]])
+    ref = attend()
+    torch.cuda.synchronize()
+    assert _bits_equal(got, ref)
