@@ -185,16 +185,18 @@ PA_API size_t pa_workspace_size_ex(int32_t num_seqs, int32_t num_tokens, int32_t
  * out: bf16 [num_tokens, num_q_heads, head_dim]; must not overlap q.  Rows
  *   that belong to no request are not written.
  * lse: fp32 [num_tokens, num_q_heads] natural-log log-sum-exp of the scaled
- *   scores, or NULL.
+ *   scores, or NULL; must not overlap q or out.
  * workspace: device memory of at least pa_workspace_size_ex(...) bytes,
- *   16-byte aligned, used only while the enqueued work runs; calls that can
- *   run concurrently need distinct workspaces.  Byte 0 holds the device status
+ *   16-byte aligned, not overlapping q, out or lse, used only while the
+ *   enqueued work runs; calls that can run concurrently need distinct
+ *   workspaces.  Byte 0 holds the device status
  *   word (PA_DEVICE_* bits), reset by every call and readable after it.
  *
  * Supported: head_dim 64 or 128, block_size 16, num_q_heads/num_kv_heads a
  * divisor of 128.  Errors: INVALID_ARG (null pointer, negative size,
- * num_q_heads % num_kv_heads != 0, bt_stride too small, out overlapping q,
- * nonzero reserved option), UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA.
+ * num_q_heads % num_kv_heads != 0, bt_stride too small, q / out / lse /
+ * workspace overlapping, nonzero reserved option), UNSUPPORTED,
+ * WORKSPACE_TOO_SMALL, CUDA.
  *
  * Concurrency inside a call: when a step can hold both prefill-shaped and
  * decode-shaped requests, the prefill kernel runs on a side stream of the

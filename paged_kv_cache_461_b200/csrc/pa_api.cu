@@ -219,11 +219,20 @@ SideStream *side_stream()
     SideStream &ss = table[dev];
     std::lock_guard<std::mutex> g(init_mu);
     if (!ss.ready) {
-        if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess)
+        if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+            // release what was created, so a later call starts from nothing instead of leaking
+            if (ss.join)
+                cudaEventDestroy(ss.join);
+            if (ss.fork)
+                cudaEventDestroy(ss.fork);
+            if (ss.stream)
+                cudaStreamDestroy(ss.stream);
+            ss.stream = nullptr;
+            ss.fork = ss.join = nullptr;
             return nullptr;
-        if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
-            return nullptr;
+        }
         ss.ready = true;
     }
     return &ss;
@@ -333,12 +342,17 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     const size_t q_bytes = (size_t)num_tokens * num_q_heads * D * 2;
     if (ranges_overlap(q, q_bytes, out, q_bytes))
         return PA_ERR_INVALID_ARG;
-    if (lse && ranges_overlap(lse, (size_t)num_tokens * num_q_heads * 4, out, q_bytes))
+    const size_t lse_bytes = lse ? (size_t)num_tokens * num_q_heads * 4 : 0;
+    if (ranges_overlap(lse, lse_bytes, out, q_bytes) || ranges_overlap(lse, lse_bytes, q, q_bytes))
         return PA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace))
         return PA_ERR_UNSUPPORTED;
     if (workspace_bytes < P.total)
         return PA_ERR_WORKSPACE_TOO_SMALL;
+    // the part of the workspace this call writes must not overlap its inputs or outputs
+    if (ranges_overlap(workspace, P.total, q, q_bytes) || ranges_overlap(workspace, P.total, out, q_bytes) ||
+        ranges_overlap(workspace, P.total, lse, lse_bytes))
+        return PA_ERR_INVALID_ARG;
 
     const int Hkv = cache->num_kv_heads;
     const bool nhd = cache->layout == PA_LAYOUT_NHD;

@@ -129,6 +129,10 @@ def test_attention_host_validation(L):
     assert _attn(L, scale=float("nan")) == 1
     assert _attn(L, out=FAKE) == 1                         # out aliases q
     assert _attn(L, out=FAKE + 100) == 1                   # partial overlap
+    assert _attn(L, lse=FAKE + 64) == 1                    # lse inside q
+    assert _attn(L, lse=FAKE + (1 << 30) + 16) == 1        # lse inside out
+    assert _attn(L, ws=FAKE - 256) == 1                    # workspace running into q
+    assert _attn(L, ws=FAKE + (1 << 30)) == 1              # workspace over out
     assert _attn(L, desc=_desc(d=256)) == 2
     assert _attn(L, hq=8 * 3) == 2                         # G = 3
     assert _attn(L, q=FAKE + 2) == 2                       # q not 16-byte aligned
