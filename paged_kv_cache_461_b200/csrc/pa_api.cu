@@ -91,8 +91,8 @@ bool make_plan(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, const 
     P.max_splits = P.NT ? (int)((msl + P.split_tokens - 1) / P.split_tokens) : 0;
     P.max_dec_units = P.NT ? (int64_t)num_seqs * P.max_splits : 0;
     P.max_pf_tiles = (int64_t)num_tokens * P.G / kPrefillRows + num_seqs + 1;
-    P.need_merge = P.NT && P.max_splits > 1;
-    const int64_t part_rows = P.need_merge ? (int64_t)num_seqs * P.QD * num_q_heads * P.max_splits : 0;
+    P.need_reduce = P.NT && P.max_splits > 1; // split partial states exist (the decode kernel merges them)
+    const int64_t part_rows = P.need_reduce ? (int64_t)num_seqs * P.QD * num_q_heads * P.max_splits : 0;
     size_t off = align_up(sizeof(WsHeader));
     P.off_dec = off;
     off = align_up(off + sizeof(int2) * (size_t)P.max_dec_units);

@@ -39,7 +39,7 @@ struct Plan {
     int64_t max_dec_units = 0;
     int64_t max_pf_tiles = 0;
     bool need_prefill = false;
-    bool need_merge = false; // split partial states exist
+    bool need_reduce = false;
     // byte offsets inside the workspace
     size_t off_dec = 0, off_pf = 0, off_red = 0, off_part_o = 0, off_part_lse = 0, total = 0;
 };
