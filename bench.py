@@ -764,8 +764,9 @@ def main():
                                  "clocks": pf_clocks}}
         line["gpu_launches"] += mx.launches_per_step * mk
 
-    if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_run(HEADLINE)
+    if ws == 1 and not args.no_cpu_baseline:
+        # the oracle on this machine's host cores, at N = 1 only (a multi-GPU run would hold every GPU meanwhile)
+        line["cpu_baseline"] = cpu_oracle_run(args.workload)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:
