@@ -250,3 +250,24 @@ def test_binding_checks_dtype_before_device(L):
     with pytest.raises(ValueError, match="block ids"):
         c.insert(h, [1])
     c.close()
+
+
+def test_boundary_from_plain_c(L, tmp_path):
+    # a C99 program includes pa.h, links libpa_b200.so and calls the host-only entry points;
+    # its chained FNV-1a digests must equal the oracle's restatement of the same definition
+    import shutil
+    from oracle import prefix as P
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(build.LIB)
+    exe = str(tmp_path / "abi_from_c")
+    subprocess.check_call([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "abi_from_c.c"), "-o", exe, "-L", libdir, "-lpa_b200",
+                           f"-Wl,-rpath,{libdir}"])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    got = r.stdout.split()
+    import numpy as np
+    want = [d.hex() for d in P.block_hashes(np.arange(48, dtype=np.int32), "fnv1a64")]
+    assert got == want
