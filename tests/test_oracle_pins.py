@@ -72,6 +72,42 @@ def test_oracle_matches_pure_python_brute_force(which):
     assert not np.isnan(out).any(), "a sentinel (unused) slot was read"
 
 
+try:
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+except ImportError:  # pragma: no cover
+    given = None
+
+
+if given is not None:
+    @settings(max_examples=150, deadline=None, derandomize=True)
+    @given(data=st.data())
+    def test_oracle_matches_brute_force_on_random_shapes(data):
+        # random request mixes (empty requests included), GQA ratios, head dims, scales and pool slack
+        R = data.draw(st.integers(1, 3))
+        ctx = [data.draw(st.integers(0, 40)) for _ in range(R)]
+        ql = [data.draw(st.integers(0, 5)) for _ in range(R)]
+        Hkv = data.draw(st.sampled_from([1, 2]))
+        G = data.draw(st.sampled_from([1, 2, 4]))
+        D = data.draw(st.sampled_from([4, 8, 16]))
+        scale = data.draw(st.floats(0.05, 1.0))
+        seed = data.draw(st.integers(0, 2 ** 31 - 1))
+        need = sum((c + q + 15) // 16 for c, q in zip(ctx, ql))
+        lay = W.build_layout("hyp", ctx, ql, num_q_heads=Hkv * G, num_kv_heads=Hkv, head_dim=D,
+                             num_blocks=need + data.draw(st.integers(0, 5)) + 1, seed=seed)
+        vals = W.make_values_numpy(lay)
+        kc, vc = _written(lay, vals)
+        out, lse, _ = oracle.attention_for(lay, kc, vc, vals.q, scale=scale)
+        bt = [list(map(int, row)) for row in lay.block_table]
+        bout, blse = brute.attention(_nested(vals.q), _nested(kc), _nested(vc), lay.query_start_loc.tolist(),
+                                     lay.seq_lens.tolist(), bt, lay.num_q_heads, lay.num_kv_heads, lay.head_dim,
+                                     scale)
+        if lay.num_tokens:
+            np.testing.assert_allclose(out, np.asarray(bout), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse, np.asarray(blse), rtol=0, atol=1e-12)
+            assert not np.isnan(out).any(), "a sentinel (unused) slot was read"
+
+
 # ----------------------------------------------------------------------------
 # closed forms
 # ----------------------------------------------------------------------------
