@@ -463,3 +463,46 @@ def test_kv_unpack_inverts_pack_and_touches_nothing_else():
     # an id outside the pool is skipped
     k3, _ = oracle.kv_unpack(st, np.array([2, -5, NB + 1], np.int32), fill, fill)
     assert np.array_equal(k3[2], k[1]) and (k3[np.arange(NB) != 2] == W.BF16_QNAN).all()
+
+
+def _brute_unpack(staging, ids, k_cache, v_cache):
+    """Pure-Python unpack: entry i's K and V overwrite block ids[i] when it is inside the pool."""
+    NB = k_cache.shape[0]
+    k2 = k_cache.reshape(NB, -1).copy()
+    v2 = v_cache.reshape(NB, -1).copy()
+    for i, b in enumerate(ids.tolist()):
+        if 0 <= b < NB:
+            k2[b] = staging[i, 0]
+            v2[b] = staging[i, 1]
+    return k2.reshape(k_cache.shape), v2.reshape(v_cache.shape)
+
+
+if given is not None:
+    @settings(max_examples=100, deadline=None, derandomize=True)
+    @given(data=st.data())
+    def test_data_movement_matches_brute_force_on_random_pools(data):
+        # random pools, random distinct slots with padding tokens, random block lists (ids outside the
+        # pool included): KV write, pack and unpack against their pure-Python restatements, bit for bit
+        seed = data.draw(st.integers(0, 2 ** 31 - 1))
+        rng = np.random.default_rng(seed)
+        NB = data.draw(st.integers(1, 9))
+        Hkv = data.draw(st.integers(1, 3))
+        D = data.draw(st.sampled_from([2, 4, 8]))
+        T = data.draw(st.integers(0, min(20, NB * 16)))
+        kc = rng.integers(0, 1 << 16, size=(NB, Hkv, 16, D), dtype=np.uint16)
+        vc = rng.integers(0, 1 << 16, size=(NB, Hkv, 16, D), dtype=np.uint16)
+        kn = rng.integers(0, 1 << 16, size=(T, Hkv, D), dtype=np.uint16)
+        vn = rng.integers(0, 1 << 16, size=(T, Hkv, D), dtype=np.uint16)
+        slots = rng.permutation(NB * 16)[:T].astype(np.int64)
+        slots[rng.random(T) < 0.25] = -1
+        a = oracle.kv_write(kn, vn, slots, kc, vc)
+        b = _brute_kv_write(kn, vn, slots, kc, vc)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+        n = data.draw(st.integers(0, 6))
+        ids = rng.integers(-2, NB + 2, size=n).astype(np.int32)
+        stg = oracle.kv_pack(kc, vc, ids)
+        assert np.array_equal(stg, _brute_pack(kc, vc, ids))
+        dst = rng.permutation(NB + 2)[:n].astype(np.int32) - 1          # distinct, some outside the pool
+        u = oracle.kv_unpack(stg, dst, kc, vc)
+        w = _brute_unpack(stg, dst, kc, vc)
+        assert np.array_equal(u[0], w[0]) and np.array_equal(u[1], w[1])
