@@ -25,13 +25,13 @@ MUTATIONS = [
      ["brute", "sdpa", "two_key", "hyp"]),
     ("gather_wrong_block", "int64_t blk = bt_row[b];", "int64_t blk = bt_row[b > 0 ? b - 1 : 0];",
      ["brute", "sdpa", "gather", "hyp"]),
-    ("merge_ignores_weights", "        z += exp(lse[s] - mx);\n", "        z += 1.0;\n", ["split"]),
+    ("merge_ignores_weights", "        z += exp(lse[s] - mx);\n", "        z += 1.0;\n", ["split", "hyp_merge"]),
     ("slot_offset_shifted", "slot_mapping[query_start_loc[r] + i] = blk * block_size + p % block_size;",
      "slot_mapping[query_start_loc[r] + i] = blk * block_size + (p + 1) % block_size;", ["slots"]),
     ("kv_write_head_stride", "int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;",
      "int64_t dst = ((blk * num_kv_heads + (num_kv_heads - 1 - h)) * block_size + off) * head_dim;",
      ["kv_write", "slots", "hyp_move"]),
-    ("lse_missing_max", "*lse = mx + log(z);", "*lse = log(z);", ["brute", "two_key", "hyp"]),
+    ("lse_missing_max", "*lse = mx + log(z);", "*lse = log(z);", ["brute", "two_key", "hyp", "hyp_merge"]),
     ("pack_k_and_v_swapped", "memcpy(dk, k_cache + b * block_elems,", "memcpy(dk, v_cache + b * block_elems,",
      ["pack", "hyp_move"]),
     ("pack_block_off_by_one", "memcpy(dv, v_cache + b * block_elems,", "memcpy(dv, v_cache + (b + 1) % num_blocks * block_elems,",
@@ -44,6 +44,7 @@ CHECKS = {
     "brute": lambda: [pins.test_oracle_matches_pure_python_brute_force(w) for w in ("micro1", "micro4")],
     "hyp": lambda: pins.test_oracle_matches_brute_force_on_random_shapes(),
     "hyp_move": lambda: pins.test_data_movement_matches_brute_force_on_random_pools(),
+    "hyp_merge": lambda: pins.test_split_merge_identity_on_random_cuts(),
     "sdpa": lambda: [pins.test_matches_torch_sdpa_on_unpaged_arrays(45, 20, 2)],
     "two_key": lambda: pins.test_hand_worked_two_key_example(),
     "split": lambda: pins.test_split_merge_reproduces_unsplit_attention(),

@@ -506,3 +506,29 @@ if given is not None:
         u = oracle.kv_unpack(stg, dst, kc, vc)
         w = _brute_unpack(stg, dst, kc, vc)
         assert np.array_equal(u[0], w[0]) and np.array_equal(u[1], w[1])
+
+
+if given is not None:
+    @settings(max_examples=100, deadline=None, derandomize=True)
+    @given(data=st.data())
+    def test_split_merge_identity_on_random_cuts(data):
+        # any cut of the keys into parts (empty parts included, in any order), attended part by part
+        # and merged, equals one pass over all keys: the identity the split-KV path relies on
+        seed = data.draw(st.integers(0, 2 ** 31 - 1))
+        rng = np.random.default_rng(seed)
+        D = data.draw(st.sampled_from([4, 16, 64]))
+        n = data.draw(st.integers(1, 200))
+        qs = data.draw(st.floats(0.1, 8.0))
+        scale = data.draw(st.floats(0.01, 1.0))
+        q = W.f32_to_bf16_bits(rng.standard_normal(D).astype(np.float32) * np.float32(qs))
+        K = W.f32_to_bf16_bits(rng.standard_normal((n, D)).astype(np.float32))
+        V = W.f32_to_bf16_bits(rng.standard_normal((n, D)).astype(np.float32))
+        full, lfull, _ = oracle.attend_dense(q, K, V, scale)
+        k = data.draw(st.integers(0, 6))
+        edges = [0] + sorted(int(x) for x in rng.integers(0, n + 1, size=k)) + [n]
+        spans = list(zip(edges[:-1], edges[1:]))
+        order = rng.permutation(len(spans))
+        parts = [oracle.attend_dense(q, K[a:b], V[a:b], scale) for a, b in (spans[i] for i in order)]
+        m, lm = oracle.merge_states(np.stack([p[0] for p in parts]), np.array([p[1] for p in parts]))
+        np.testing.assert_allclose(m, full, rtol=0, atol=1e-12)
+        assert abs(lm - lfull) < 1e-10
