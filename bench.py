@@ -759,6 +759,8 @@ def main():
             "prefill_flops_per_step": mx.prefill_flops,
             "prefill_roofline": {"bound": "tensor", "achieved": pf_tf, "peak": peaks["bf16_tflops"],
                                  "unit": "TFLOP/s", "frac": pf_tf / peaks["bf16_tflops"], "ms_per_launch": pf_ms,
+                                 "sustained_peak": peaks["bf16_tflops_sustained"],
+                                 "frac_of_sustained": pf_tf / peaks["bf16_tflops_sustained"],
                                  "kernel": "pa_attention_mixed on the prefill chunks alone, prefill-only mode (plan + prefill_kernel)",
                                  "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                                  "clocks": pf_clocks}}
