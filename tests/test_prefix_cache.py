@@ -181,3 +181,56 @@ def test_prefix_hash_argument_checks():
     assert L.pa_prefix_block_hashes(toks.ctypes.data, 15, None, 0, None, ctypes.byref(n)) == 0 and n.value == 0
     assert L.pa_prefix_cache_longest_hit(None, None, 0, None) == -1
     assert L.pa_prefix_cache_size(None) == -1
+
+
+# ----------------------------------------------------------------------------- random operation sequences
+
+from hypothesis import settings as _settings
+from hypothesis import strategies as _st
+from hypothesis.stateful import RuleBasedStateMachine, invariant, rule
+
+
+class PrefixCacheMachine(RuleBasedStateMachine):
+    """Random inserts, block removals and lookups against a plain model: a dict from digest to block
+    where the first mapping of a digest wins and a block holds at most one digest."""
+
+    def __init__(self):
+        super().__init__()
+        self.cache = api.PrefixCache()
+        self.model = {}
+        # three prompts that share prefixes of different lengths, hashed once
+        base = np.arange(16 * 6, dtype=np.int32)
+        self.prompts = [api.prefix_block_hashes(base),
+                        api.prefix_block_hashes(np.concatenate([base[:48], base[48:] + 1000])),
+                        api.prefix_block_hashes(np.concatenate([base[:16], base[16:] + 2000]))]
+
+    def teardown(self):
+        self.cache.close()
+
+    @rule(p=_st.integers(0, 2), n=_st.integers(0, 6), first=_st.integers(0, 40))
+    def insert(self, p, n, first):
+        h = self.prompts[p][:n]
+        ids = np.arange(first, first + len(h), dtype=np.int32)
+        self.cache.insert(h, ids)
+        for d, b in zip((bytes(x) for x in h), ids.tolist()):
+            if d not in self.model and b not in self.model.values():
+                self.model[d] = b
+
+    @rule(b=_st.integers(0, 46))
+    def remove(self, b):
+        self.cache.remove_block(b)
+        self.model = {d: v for d, v in self.model.items() if v != b}
+
+    @rule(p=_st.integers(0, 2))
+    def lookup(self, p):
+        h = self.prompts[p]
+        assert self.cache.longest_hit(h).tolist() == P.longest_hit_brute(self.model, [bytes(x) for x in h])
+
+    @invariant()
+    def same_size(self):
+        assert len(self.cache) == len(self.model)
+
+
+TestPrefixCacheMachine = PrefixCacheMachine.TestCase
+TestPrefixCacheMachine.settings = _settings(max_examples=60, stateful_step_count=30, deadline=None,
+                                            derandomize=True)
