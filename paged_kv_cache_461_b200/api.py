@@ -119,9 +119,18 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
-def _stream(stream=None):
+def _stream(stream=None, device: Optional[torch.device] = None):
+    """The stream to enqueue on: torch's current stream unless one is given.  The library launches on
+    the current CUDA device, so that device (and a given stream's) must be the tensors' device."""
+    if device is not None:
+        cur = torch.cuda.current_device()
+        if device.index != cur:
+            raise ValueError(f"the tensors are on {device} but the current CUDA device is cuda:{cur} "
+                             f"(call under torch.cuda.device({device.index}))")
     if stream is None:
         stream = torch.cuda.current_stream()
+    elif device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -221,7 +230,7 @@ def kv_write(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tenso
     T = k_new.shape[0]
     _need(slot_mapping, torch.int64, "slot_mapping", shape=(T,), dense=True, device=k_cache.device)
     _check(lib().pa_kv_write(_ptr(k_new), _ptr(v_new), row_stride, _ptr(slot_mapping), T, _ptr(k_cache),
-                             _ptr(v_cache), ctypes.byref(d), _stream(stream)), "pa_kv_write")
+                             _ptr(v_cache), ctypes.byref(d), _stream(stream, k_cache.device)), "pa_kv_write")
 
 
 def build_slot_mapping(query_start_loc: torch.Tensor, seq_lens: torch.Tensor, block_table: torch.Tensor,
@@ -232,7 +241,7 @@ def build_slot_mapping(query_start_loc: torch.Tensor, seq_lens: torch.Tensor, bl
     _need(out, torch.int64, "out", shape=(num_tokens,), dense=True, device=query_start_loc.device)
     _check(lib().pa_build_slot_mapping(_ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
                                        block_table.stride(0), seq_lens.shape[0], num_tokens, _ptr(out),
-                                       _stream(stream)), "pa_build_slot_mapping")
+                                       _stream(stream, query_start_loc.device)), "pa_build_slot_mapping")
     return out
 
 
@@ -279,7 +288,7 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
                                        block_table.stride(0), R, T, int(max_query_len), int(max_seq_len),
                                        float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(),
-                                       ctypes.byref(o) if o else None, _stream(stream)), "pa_attention_mixed")
+                                       ctypes.byref(o) if o else None, _stream(stream, q.device)), "pa_attention_mixed")
     return out
 
 
@@ -305,7 +314,7 @@ def attention_mixed_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
                                             _ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
                                             block_table.stride(0), R, T, int(max_query_len), int(max_seq_len),
                                             float(softmax_scale), _ptr(out), _ptr(lse),
-                                            ctypes.byref(o) if o else None, _stream(stream)),
+                                            ctypes.byref(o) if o else None, _stream(stream, q.device)),
            "pa_attention_mixed_noalloc")
     return out
 
@@ -341,7 +350,7 @@ def attention_decode_fused(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Te
                                            _ptr(block_table), block_table.stride(0), R, T, int(max_query_len),
                                            int(max_seq_len), float(softmax_scale), _ptr(out), _ptr(lse),
                                            _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                           ctypes.byref(o) if o else None, _stream(stream)),
+                                           ctypes.byref(o) if o else None, _stream(stream, q.device)),
            "pa_attention_decode_fused")
     return out
 
@@ -358,7 +367,7 @@ def kv_pack(k_cache: torch.Tensor, v_cache: torch.Tensor, block_ids: torch.Tenso
         staging = torch.empty((n, 2, elems), dtype=k_cache.dtype, device=k_cache.device)
     _need(staging, torch.bfloat16, "staging", shape=(n, 2, elems), dense=True, device=k_cache.device)
     _check(lib().pa_kv_pack(_ptr(k_cache), _ptr(v_cache), ctypes.byref(d), _ptr(block_ids), n, _ptr(staging),
-                            _stream(stream)), "pa_kv_pack")
+                            _stream(stream, k_cache.device)), "pa_kv_pack")
     return staging
 
 
@@ -372,7 +381,7 @@ def kv_unpack(staging: torch.Tensor, block_ids: torch.Tensor, k_cache: torch.Ten
     _need(staging, torch.bfloat16, "staging", shape=(n, 2, d.num_kv_heads * d.block_size * d.head_dim), dense=True,
           device=k_cache.device)
     _check(lib().pa_kv_unpack(_ptr(staging), _ptr(block_ids), block_ids.shape[0], _ptr(k_cache), _ptr(v_cache),
-                              ctypes.byref(d), _stream(stream)), "pa_kv_unpack")
+                              ctypes.byref(d), _stream(stream, k_cache.device)), "pa_kv_unpack")
 
 
 def merge_attn_states(part_out: torch.Tensor, part_lse: torch.Tensor, parts_per_row: Optional[torch.Tensor] = None,
@@ -393,7 +402,7 @@ def merge_attn_states(part_out: torch.Tensor, part_lse: torch.Tensor, parts_per_
     if lse_out is not None:
         _need(lse_out, torch.float32, "lse_out", shape=(N, H), dense=True, device=dev)
     _check(lib().pa_merge_attn_states(_ptr(part_out), _ptr(part_lse), _ptr(parts_per_row), N, H, S, D, _ptr(out),
-                                      _ptr(lse_out), _stream(stream)), "pa_merge_attn_states")
+                                      _ptr(lse_out), _stream(stream, dev)), "pa_merge_attn_states")
     return out
 
 
@@ -406,7 +415,7 @@ def debug_gather_kv(cache: torch.Tensor, bt_row: torch.Tensor, seq_len: int, str
         raise ValueError("bt_row holds fewer block ids than seq_len needs")
     out = torch.empty((seq_len, d.num_kv_heads, d.head_dim), dtype=cache.dtype, device=cache.device)
     _check(lib().pa_debug_gather_kv(_ptr(cache), ctypes.byref(d), _ptr(bt_row), seq_len, _ptr(out),
-                                    _stream(stream)), "pa_debug_gather_kv")
+                                    _stream(stream, cache.device)), "pa_debug_gather_kv")
     return out
 
 

@@ -271,3 +271,23 @@ def test_boundary_from_plain_c(L, tmp_path):
     import numpy as np
     want = [d.hex() for d in P.block_hashes(np.arange(48, dtype=np.int32), "fnv1a64")]
     assert got == want
+
+
+def test_binding_launches_only_on_the_tensors_device(monkeypatch):
+    # the library launches on the current CUDA device: tensors (or a given stream) on another device
+    # are refused before the call; stand-ins replace torch.cuda's device and stream queries
+    import torch
+
+    class Stream:
+        def __init__(self, dev, handle):
+            self.device, self.cuda_stream = dev, handle
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda: Stream(torch.device("cuda", 0), 1234))
+    cuda0, cuda1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    assert api._stream(None, cuda0).value == 1234
+    assert api._stream(Stream(cuda0, 99), cuda0).value == 99
+    with pytest.raises(ValueError, match="current CUDA device"):
+        api._stream(None, cuda1)
+    with pytest.raises(ValueError, match="stream is on"):
+        api._stream(Stream(cuda1, 5), cuda0)
