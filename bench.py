@@ -20,6 +20,7 @@ a bounded sample of the same workload (the only reference this method has).
 from __future__ import annotations
 
 import argparse
+import atexit
 import hashlib
 import json
 import math
@@ -88,11 +89,21 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", str(period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            atexit.register(self._kill)  # never leave the sampler running if the bench ends early
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
             self.first.wait(timeout=5.0)
         except OSError:
             self.proc = None
+
+    def _kill(self):
+        p = self.proc
+        if p is not None and p.poll() is None:
+            p.terminate()
+            try:
+                p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                p.kill()
 
     def _read(self):
         for line in self.proc.stdout:
@@ -105,11 +116,7 @@ class ClockSampler:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         time.sleep(0.05)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+        self._kill()
         self.t.join(timeout=2)
         inside = [r for ts, r in self.rows if t0 <= ts <= t1 + 0.02]
         note = "samples inside the timed region"

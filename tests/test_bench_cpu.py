@@ -44,3 +44,31 @@ def test_reference_arm_other_ranks_exit_without_work():
 def test_fewer_than_three_warmups_are_refused():
     r = _bench("--impl", "reference", "--steps", "3", "--warmup", "2")
     assert r.returncode != 0 and "warm-up" in r.stderr
+
+
+def test_clock_sampler_always_ends_its_child():
+    # stop() (and the exit hook) end the background sampler process; a stand-in child replaces nvidia-smi
+    import shutil
+    import threading
+
+    import bench
+    if shutil.which("sleep") is None:
+        return
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.rows, s.first = [], threading.Event()
+    s.proc = subprocess.Popen(["sleep", "30"], stdout=subprocess.PIPE, text=True)
+    s.t = threading.Thread(target=s._read, daemon=True)
+    s.t.start()
+    r = s.stop(0.0, 1.0)
+    assert s.proc.poll() is not None and r["samples"] == 0
+    s._kill()                                            # a second end is harmless
+
+
+def test_clock_sampler_without_nvidia_smi_reports_it():
+    import shutil
+
+    import bench
+    if shutil.which("nvidia-smi") is not None:
+        return
+    r = bench.ClockSampler(0).stop(0.0, 1.0)
+    assert r["reasons"] == ["nvidia-smi unavailable"] and r["samples"] == 0
