@@ -15,32 +15,34 @@
 // item to the next, so the next item's Q load and first QK^T overlap the
 // previous item's last steps and epilogue.
 //
-// Warp roles (576 threads, one CTA per SM):
-//   warp 0      TMA producer: per item both Q tiles (3-D boxes {64 d, G heads,
-//               128/G tokens}, 128-byte swizzle) once the previous item's last
-//               QK^T is done, then per 128-key step the K tile and the V tile (8
-//               paged blocks x 64-column halves, 2-D boxes) into separate
-//               2-stage rings;
-//   warp 1      TMEM allocation (512 columns: S_A, O_A, S_B, O_B) and the MMAs
-//               (one elected lane issues, the warp stays converged), in the order
+// Warpgroup roles (512 threads, one CTA per SM; registers moved between the
+// warpgroups with setmaxnreg so that a softmax thread can hold a whole row):
+//   WG 0, WG 1  softmax of tile A and of tile B: one thread per query row
+//               (= TMEM lane), all 128 scores of a key step in registers after
+//               one tcgen05.ld pass.  Causal mask by select, row max over the
+//               thread's own registers, P = exp2(s*c - m*c) with packed fp32x2
+//               FMAs, bf16 P back into TMEM over S with tcgen05.st.  O is
+//               rescaled in TMEM only when a row's max grows by more than 2^8
+//               (a stale max leaves the normalised result unchanged).  After a
+//               tile's last step the row sum and max go to the epilogue
+//               warpgroup through shared memory and the softmax moves straight
+//               on to its next item.
+//   WG 2        epilogue of both tiles: waits for a tile's final O, writes O / l
+//               as bf16 (and the LSE), then frees O for the next item's first PV.
+//   WG 3        warp 12: TMA producer -- per item both Q tiles (3-D boxes
+//               {64 d, G heads, 128/G tokens}, 128-byte swizzle) once the
+//               previous item's last QK^T is done, then per 128-key step the K
+//               tile and the V tile (8 paged blocks x 64-column halves, 2-D
+//               boxes) into separate 2-stage rings;
+//               warp 13: TMEM allocation (512 columns: S_A, O_A, S_B, O_B) and
+//               the MMAs (one elected lane issues, the warp stays converged), in
+//               the order
 //                 PV_A(j-1), S_A(j), PV_B(j-1), S_B(j)   (ping-pong)
 //               so the tensor core works on one tile while the other tile's
 //               softmax runs.  S = Q K^T is SS (both operands in smem);
 //               O += P V reads P from TMEM (written over S by the softmax) and V
 //               from smem as an MN-major operand.  Each group of 8 MMAs is
-//               issued from one asm block with prebuilt descriptors;
-//   warps 2..9  softmax of tile A, warps 10..17 softmax of tile B: each query
-//               row (= TMEM lane) is shared by two threads in two warps of the
-//               same TMEM lane quadrant, one per 64-key half, so a thread holds
-//               its 64 scores in registers after one tcgen05.ld pass.  Causal
-//               mask by select, row max exchanged between the two halves
-//               through shared memory (64-thread named barrier),
-//               P = exp2(s*c - m*c) with packed fp32x2 FMAs, bf16 P back into
-//               TMEM over S with tcgen05.st; O is rescaled in TMEM only when a
-//               row's max grows by more than 2^8 (a stale max leaves the
-//               normalised result unchanged); the epilogue writes O / l as
-//               bf16, each thread half of the head dimension, then frees O for
-//               the next item.
+//               issued from one asm block with prebuilt descriptors.
 // Ordering facts the pipeline relies on: a commit fires only once every
 // earlier MMA of the issuing thread is done, so when the softmax sees S_X(j)
 // the previous PV_X(j-1) has finished with P_X and O_X; and MMAs issued by one
@@ -71,11 +73,9 @@ struct PfCfg {
     static constexpr int kOffV = kOffK + kStages * kTile; // V ring
     static constexpr int kOffBar = kOffV + kStages * kTile;
     static constexpr int kBarBytes = 256;
-    static constexpr int kOffX = kOffBar + kBarBytes;  // per-step row-max exchange: [tile][parity][half][128] fp32
-    static constexpr int kXBytes = 2 * 2 * 2 * 128 * 4;
-    static constexpr int kOffL = kOffX + kXBytes;      // epilogue row-sum exchange: [tile][half][128] fp32
-    static constexpr int kLBytes = 2 * 2 * 128 * 4;
-    static constexpr int kUsed = kOffL + kLBytes + 1024;
+    static constexpr int kOffLM = kOffBar + kBarBytes; // row sum and max for the epilogue: [tile][item parity][l|m][128] fp32
+    static constexpr int kLMBytes = 2 * 2 * 2 * 128 * 4;
+    static constexpr int kUsed = kOffLM + kLMBytes + 1024;
     // keep one CTA per SM (each CTA allocates all 512 TMEM columns)
     static constexpr int kSmem = kUsed > 120 * 1024 ? kUsed : 120 * 1024;
 };
@@ -92,17 +92,26 @@ enum PfBar {
     B_VF = 6,    // 2: V stage full
     B_VE = 8,    // 2: V stage consumed
     B_SF = 10,   // 2: S_X ready (per tile)
-    B_PF = 12,   // 2: P_X written (per tile, 256 arrivals)
+    B_PF = 12,   // 2: P_X written (per tile, one arrival per row)
     B_OF = 14,   // 2: O_X of an item final (per tile)
-    B_OE = 16,   // 2: O_X of an item read by the epilogue (per tile, 256 arrivals)
-    B_VFIX = 18, // V tail of an item zeroed
-    B_FIN = 19,
-    B_NUM = 20
+    B_OE = 16,   // 2: O_X of an item read by the epilogue (per tile, one arrival per row)
+    B_LF = 18,   // 2: row sums and maxima of an item's tile X in shared memory (one arrival per row)
+    B_VFIX = 20, // V tail of an item zeroed
+    B_FIN = 21,
+    B_NUM = 22
 };
 
 constexpr uint32_t kTmemCols = 512;
-constexpr int kThreads = 576;
-constexpr int kSoftmaxThreads = 256; // per tile: 128 rows x 2 halves
+constexpr int kThreads = 512;
+constexpr int kRowThreads = 128; // one thread per query row of a tile
+// Registers per thread of each warpgroup after the split (the launch gives every thread
+// 65536 / 512 = 128): two softmax warpgroups hold a whole 128-key row of scores, the
+// epilogue and control warpgroups need little.
+constexpr int kRegSoftmax = 176;
+constexpr int kRegEpilogue = 80;
+constexpr int kRegControl = 72;
+constexpr int kRegSplit = kRowThreads * (2 * kRegSoftmax + kRegEpilogue + kRegControl);
+static_assert(kRegSplit <= 65536, "the warpgroup budgets must fit the CTA's register pool");
 
 struct TileGeo {
     int rows;  // valid query rows (0 = tile absent)
@@ -186,10 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const uint32_t bar = sbase + Cfg::kOffBar;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffBar + B_NUM * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffBar + B_NUM * 8 + 4);
+    float *lm_all = reinterpret_cast<float *>(smem + Cfg::kOffLM);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wg = warp >> 2;
     const int G = p.G;
     const int TQ = kPrefillRows / G; // tokens per 128-row tile
+    constexpr int kProducerWarp = 12, kMmaWarp = 13;
 
     // ---- setup: barriers, TMEM
     if (threadIdx.x == 0) {
@@ -201,16 +213,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             mbar_init(bar + (B_VF + s) * 8, 1);
             mbar_init(bar + (B_VE + s) * 8, 1);
             mbar_init(bar + (B_SF + s) * 8, 1);
-            mbar_init(bar + (B_PF + s) * 8, kSoftmaxThreads);
+            mbar_init(bar + (B_PF + s) * 8, kRowThreads);
             mbar_init(bar + (B_OF + s) * 8, 1);
-            mbar_init(bar + (B_OE + s) * 8, kSoftmaxThreads);
+            mbar_init(bar + (B_OE + s) * 8, kRowThreads);
+            mbar_init(bar + (B_LF + s) * 8, kRowThreads);
         }
         mbar_init(bar + B_VFIX * 8, 1);
         mbar_init(bar + B_FIN * 8, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
@@ -224,112 +237,113 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         atomicOr(&p.hdr->status, PA_DEVICE_WAIT_TIMEOUT);
     };
 
-    if (warp == 0) {
-        // ===================================================== TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-        }
-        bool ok = true;
-        uint32_t gs = 0; // K/V steps loaded so far by this CTA
-        uint32_t nq = 0; // items whose Q was loaded
-        for (int k = 0, item = snake_item(0, n_ctas); ok && item < n_items; item = snake_item(++k, n_ctas)) {
-            const ItemGeo g = item_geo(p, item);
-            // Q of this item, once the previous item's last QK^T has read the old Q
-            if (nq > 0 && !mbar_wait_warp(bar + B_QE * 8, (nq - 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
+    if (wg == 3) {
+        wg_reg_lower<kRegControl>();
+        if (warp == kProducerWarp) {
+            // ===================================================== TMA producer
             if (lane == 0) {
-                const int ntiles = g.t1.rows ? 2 : 1;
-                mbar_arrive_expect_tx(bar + B_Q * 8, ntiles * Cfg::kTile);
-                for (int x = 0; x < ntiles; ++x)
-#pragma unroll
-                    for (int hf = 0; hf < Cfg::kHalves; ++hf)
-                        tma_load_3d(sQ + x * Cfg::kTile + hf * Cfg::kHalfBytes, &tm_q, hf * 64, g.h * G,
-                                    g.qs + g.tok0 + x * TQ, bar + B_Q * 8);
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
             }
-            ++nq;
-            const int32_t *bt_row = p.bt + (int64_t)g.r * p.bt_stride;
-            for (int j = 0; j < g.n_steps; ++j, ++gs) {
-                const int st = gs & 1;
-                const int nblk = blocks_in_step(g.n_keys_all, j);
-                // HND: 2-D map, row (bid*Hkv + h)*16;  NHD: 3-D map, (head h, token row bid*16)
-                int y = -kBlockSize; // out-of-bounds box: TMA fills zeros
-                if (lane < nblk) {
-                    const int bid = bt_row[j * kStepBlocks + lane];
-                    if ((unsigned)bid < (unsigned long long)p.num_blocks)
-                        y = (p.nhd ? bid : bid * p.Hkv + g.h) * kBlockSize;
-                    else
-                        atomicOr(&p.hdr->status, PA_DEVICE_BAD_BLOCK);
-                }
-                const uint32_t tx = (uint32_t)(nblk * kBlockSize * D * 2);
-                const uint32_t ph_prev = ((gs >> 1) - 1) & 1; // phase of this stage's previous use
-                // K into stage st once the K two steps back is consumed
-                if (gs >= 2 && !mbar_wait_warp(bar + (B_KE + st) * 8, ph_prev, abort_flag)) {
+            bool ok = true;
+            uint32_t gs = 0; // K/V steps loaded so far by this CTA
+            uint32_t nq = 0; // items whose Q was loaded
+            for (int k = 0, item = snake_item(0, n_ctas); ok && item < n_items; item = snake_item(++k, n_ctas)) {
+                const ItemGeo g = item_geo(p, item);
+                // Q of this item, once the previous item's last QK^T has read the old Q
+                if (nq > 0 && !mbar_wait_warp(bar + B_QE * 8, (nq - 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                if (lane == 0)
-                    mbar_arrive_expect_tx(bar + (B_KF + st) * 8, tx);
-                __syncwarp();
-                if (lane < nblk)
+                if (lane == 0) {
+                    const int ntiles = g.t1.rows ? 2 : 1;
+                    mbar_arrive_expect_tx(bar + B_Q * 8, ntiles * Cfg::kTile);
+                    for (int x = 0; x < ntiles; ++x)
 #pragma unroll
-                    for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-                        const uint32_t dst = sK0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128);
-                        if (p.nhd)
-                            tma_load_3d(dst, &tm_k, hf * 64, g.h, y, bar + (B_KF + st) * 8);
-                        else
-                            tma_load_2d(dst, &tm_k, hf * 64, y, bar + (B_KF + st) * 8);
-                    }
-                // V into stage st once the V two steps back is consumed
-                if (gs >= 2 && !mbar_wait_warp(bar + (B_VE + st) * 8, ph_prev, abort_flag)) {
-                    ok = false;
-                    break;
+                        for (int hf = 0; hf < Cfg::kHalves; ++hf)
+                            tma_load_3d(sQ + x * Cfg::kTile + hf * Cfg::kHalfBytes, &tm_q, hf * 64, g.h * G,
+                                        g.qs + g.tok0 + x * TQ, bar + B_Q * 8);
                 }
-                if (lane == 0)
-                    mbar_arrive_expect_tx(bar + (B_VF + st) * 8, tx);
-                __syncwarp();
-                if (lane < nblk)
-#pragma unroll
-                    for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-                        const uint32_t dst = sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128);
-                        if (p.nhd)
-                            tma_load_3d(dst, &tm_v, hf * 64, g.h, y, bar + (B_VF + st) * 8);
+                ++nq;
+                const int32_t *bt_row = p.bt + (int64_t)g.r * p.bt_stride;
+                for (int j = 0; j < g.n_steps; ++j, ++gs) {
+                    const int st = gs & 1;
+                    const int nblk = blocks_in_step(g.n_keys_all, j);
+                    // HND: 2-D map, row (bid*Hkv + h)*16;  NHD: 3-D map, (head h, token row bid*16)
+                    int y = -kBlockSize; // out-of-bounds box: TMA fills zeros
+                    if (lane < nblk) {
+                        const int bid = bt_row[j * kStepBlocks + lane];
+                        if ((unsigned)bid < (unsigned long long)p.num_blocks)
+                            y = (p.nhd ? bid : bid * p.Hkv + g.h) * kBlockSize;
                         else
-                            tma_load_2d(dst, &tm_v, hf * 64, y, bar + (B_VF + st) * 8);
+                            atomicOr(&p.hdr->status, PA_DEVICE_BAD_BLOCK);
                     }
-                if (g.tail_fix && j == g.n_steps - 1) {
-                    // zero the V rows past the end of the sequence in its last block
-                    if (!mbar_wait_warp(bar + (B_VF + st) * 8, (gs >> 1) & 1, abort_flag)) {
+                    const uint32_t tx = (uint32_t)(nblk * kBlockSize * D * 2);
+                    const uint32_t ph_prev = ((gs >> 1) - 1) & 1; // phase of this stage's previous use
+                    // K into stage st once the K two steps back is consumed
+                    if (gs >= 2 && !mbar_wait_warp(bar + (B_KE + st) * 8, ph_prev, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const int lb = (g.L - 1) / kBlockSize - j * kStepBlocks;
-                    const int first = g.L % kBlockSize;
-                    const int nrow = kBlockSize - first;
-                    const int nz = nrow * Cfg::kHalves * 8; // 16-byte chunks
-                    for (int i = lane; i < nz; i += 32) {
-                        const int chunk = i & 7;
-                        const int rr = (i >> 3) % nrow;
-                        const int hf = (i >> 3) / nrow;
-                        const uint32_t addr = sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes +
-                                              (lb * kBlockSize + first + rr) * 128 + chunk * 16;
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
                     if (lane == 0)
-                        mbar_arrive(bar + B_VFIX * 8);
+                        mbar_arrive_expect_tx(bar + (B_KF + st) * 8, tx);
+                    __syncwarp();
+                    if (lane < nblk)
+#pragma unroll
+                        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+                            const uint32_t dst = sK0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128);
+                            if (p.nhd)
+                                tma_load_3d(dst, &tm_k, hf * 64, g.h, y, bar + (B_KF + st) * 8);
+                            else
+                                tma_load_2d(dst, &tm_k, hf * 64, y, bar + (B_KF + st) * 8);
+                        }
+                    // V into stage st once the V two steps back is consumed
+                    if (gs >= 2 && !mbar_wait_warp(bar + (B_VE + st) * 8, ph_prev, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(bar + (B_VF + st) * 8, tx);
+                    __syncwarp();
+                    if (lane < nblk)
+#pragma unroll
+                        for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+                            const uint32_t dst = sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes + lane * (kBlockSize * 128);
+                            if (p.nhd)
+                                tma_load_3d(dst, &tm_v, hf * 64, g.h, y, bar + (B_VF + st) * 8);
+                            else
+                                tma_load_2d(dst, &tm_v, hf * 64, y, bar + (B_VF + st) * 8);
+                        }
+                    if (g.tail_fix && j == g.n_steps - 1) {
+                        // zero the V rows past the end of the sequence in its last block
+                        if (!mbar_wait_warp(bar + (B_VF + st) * 8, (gs >> 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const int lb = (g.L - 1) / kBlockSize - j * kStepBlocks;
+                        const int first = g.L % kBlockSize;
+                        const int nrow = kBlockSize - first;
+                        const int nz = nrow * Cfg::kHalves * 8; // 16-byte chunks
+                        for (int i = lane; i < nz; i += 32) {
+                            const int chunk = i & 7;
+                            const int rr = (i >> 3) % nrow;
+                            const int hf = (i >> 3) / nrow;
+                            const uint32_t addr = sV0 + st * Cfg::kTile + hf * Cfg::kHalfBytes +
+                                                  (lb * kBlockSize + first + rr) * 128 + chunk * 16;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(bar + B_VFIX * 8);
+                    }
                 }
             }
-        }
-        if (!ok && lane == 0)
-            fail();
-    } else if (warp == 1) {
-        // ===================================================== MMA issuer (whole warp, one elected lane issues)
-        {
+            if (!ok && lane == 0)
+                fail();
+        } else if (warp == kMmaWarp) {
+            // ===================================================== MMA issuer (whole warp, one elected lane issues)
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kStepKeys, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             // Descriptors are built once; per MMA only the 14-bit start-address field moves, by a
@@ -460,18 +474,75 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             umma_commit(bar + B_FIN * 8);
             (void)mbar_wait_warp(bar + B_FIN * 8, 0);
         }
-    } else {
-        // ===================================================== softmax / epilogue (warps 2..9: A, 10..17: B)
-        const int x = (warp - 2) >> 3;          // tile
-        const int half = ((warp - 2) >> 2) & 1; // 64-key half of the row (and half of the head dim)
+    } else if (wg == 2) {
+        // ===================================================== epilogue of both tiles
+        wg_reg_lower<kRegEpilogue>();
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-        const int row = quad * 32 + lane;       // query row of the tile = TMEM lane
+        const int row = threadIdx.x & 127;      // query row of the tile = TMEM lane
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        const float c = p.scale_log2;
+        bool ok = true;
+        uint32_t titem[2] = {0, 0};
+        for (int k = 0, item = snake_item(0, n_ctas); ok && item < n_items; item = snake_item(++k, n_ctas)) {
+            const ItemGeo gi = item_geo(p, item);
+            for (int x = 0; x < 2; ++x) {
+                const TileGeo g = x ? gi.t1 : gi.t0;
+                if (g.rows == 0)
+                    continue;
+                if (!mbar_wait_warp(bar + (B_LF + x) * 8, titem[x] & 1, abort_flag) ||
+                    !mbar_wait_warp(bar + (B_OF + x) * 8, titem[x] & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float *slot = lm_all + x * 512 + (titem[x] & 1) * 256;
+                const float l_sum = slot[row], m_ref = slot[128 + row];
+                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const bool store = row < g.rows;
+                const int t = gi.qs + gi.tok0 + x * TQ + row / G;
+                const int hq = gi.h * G + row % G;
+                __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D;
+                const uint32_t tO = tmem + lane_addr + col_o(x);
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32p(tO + cc * 32, o);
+                    tmem_wait_ld();
+                    if (cc == D / 32 - 1) {
+                        // O_X may now be overwritten by the next item's first PV
+                        tc_fence_before();
+                        mbar_arrive(bar + (B_OE + x) * 8);
+                    }
+                    if (store) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+                            v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                            v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+                            v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+                            *reinterpret_cast<uint4 *>(dst + cc * 32 + i) = v;
+                        }
+                    }
+                }
+                ++titem[x];
+                if (store && p.lse)
+                    p.lse[(int64_t)t * p.Hq + hq] =
+                        l_sum > 0.f ? (m_ref * c + log2f(l_sum)) * 0.69314718055994531f : -CUDART_INF_F;
+            }
+        }
+        if (!ok && lane == 0)
+            fail();
+    } else {
+        // ===================================================== softmax (WG 0: tile A, WG 1: tile B)
+        wg_reg_raise<kRegSoftmax>();
+        const int x = wg;
+        const int quad = warp & 3;              // TMEM lane quadrant this warp may access
+        const int row = threadIdx.x & 127;      // query row of the tile = TMEM lane
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         const uint32_t tS = tmem + lane_addr + col_s(x);
-        const uint32_t tO = tmem + lane_addr + col_o(x) + half * (D / 2);
-        const int bar_id = 1 + x * 4 + quad; // named barrier of the two warps sharing these rows
-        float *xch = reinterpret_cast<float *>(smem + Cfg::kOffX) + x * (2 * 2 * 128);
-        float *lch = reinterpret_cast<float *>(smem + Cfg::kOffL) + x * (2 * 128);
+        const uint32_t tO = tmem + lane_addr + col_o(x);
+        float *lm = lm_all + x * 512;
         const float c = p.scale_log2;
         const float thresh = 8.f / c; // 2^8 growth, in raw score units
         bool ok = true;
@@ -482,39 +553,40 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             if (g.rows == 0)
                 continue;
             const int p_row = row < g.rows ? g.p_min + row / G : g.p_max;
-            float m_ref = -CUDART_INF_F;     // reference max, raw score units (same in both halves)
-            uint64_t l2 = f2_pack(0.f, 0.f); // exact fp32 partial row sum of this half
+            float m_ref = -CUDART_INF_F;      // reference max, raw score units
+            uint64_t l2a = f2_pack(0.f, 0.f); // exact fp32 row sum, two packed chains
+            uint64_t l2b = f2_pack(0.f, 0.f);
             for (int j = 0; j < g.nkt; ++j, ++tstep) {
                 if (!mbar_wait_warp(bar + (B_SF + x) * 8, tstep & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int key0 = j * kStepKeys + half * 64;
-                const bool diag = j * kStepKeys + kStepKeys - 1 > g.p_min; // causal mask needed
-                uint32_t sv[64];
-                tmem_ld32p(tS + half * 64, sv);
-                tmem_ld32p(tS + half * 64 + 32, sv + 32);
+                const int key0 = j * kStepKeys;
+                const bool diag = key0 + kStepKeys - 1 > g.p_min; // causal mask needed
+                uint32_t sv[128];
+                tmem_ld32p(tS, sv);
+                tmem_ld32p(tS + 32, sv + 32);
+                tmem_ld32p(tS + 64, sv + 64);
+                tmem_ld32p(tS + 96, sv + 96);
                 tmem_wait_ld();
                 if (diag) {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
+                    for (int i = 0; i < 128; ++i)
                         if (key0 + i > p_row)
                             sv[i] = __float_as_uint(-CUDART_INF_F);
                 }
-                // row max: four independent chains, then combined
-                float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+                // row max: eight independent chains, then combined
+                float m8[8];
 #pragma unroll
-                for (int i = 0; i < 64; i += 8)
+                for (int q = 0; q < 8; ++q)
+                    m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        m4[q4] = fmax3(m4[q4], __uint_as_float(sv[i + 2 * q4]), __uint_as_float(sv[i + 2 * q4 + 1]));
-                float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                // combine with the other half of the row (double-buffered by step parity)
-                float *slot = xch + (tstep & 1) * 256;
-                slot[half * 128 + row] = mx;
-                asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-                mx = fmaxf(mx, slot[(half ^ 1) * 128 + row]);
+                for (int i = 16; i < 128; i += 16)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        m8[q] = fmax3(m8[q], __uint_as_float(sv[i + 2 * q]), __uint_as_float(sv[i + 2 * q + 1]));
+                const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
                 float alpha = 1.f;
                 if (j == 0) {
                     m_ref = mx;
@@ -522,15 +594,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     alpha = fast_exp2((m_ref - mx) * c);
                     m_ref = mx;
                 }
-                l2 = f2_mul(l2, f2_pack(alpha, alpha));
-                // P = exp2(s*c - m*c) -> bf16 pairs -> TMEM columns [32*half, 32*half + 32) of S_X.
-                // Both halves finished reading S before the barrier above.
+                const uint64_t a2 = f2_pack(alpha, alpha);
+                l2a = f2_mul(l2a, a2);
+                l2b = f2_mul(l2b, a2);
+                // P = exp2(s*c - m*c) -> bf16 pairs -> TMEM columns [0, 64) of S_X (all of S was read above)
                 const uint64_t c2 = f2_pack(c, c);
                 const float nm = -m_ref * c;
                 const uint64_t nm2 = f2_pack(nm, nm);
-                uint64_t lb2 = f2_pack(0.f, 0.f); // second row-sum chain
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
+                for (int cc = 0; cc < 4; ++cc) {
                     uint32_t w[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
@@ -541,26 +613,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                                   e0, e1);
                         const float p0 = fast_exp2(e0), p1 = fast_exp2(e1);
                         if (i & 1)
-                            lb2 = f2_add(lb2, f2_pack(p0, p1));
+                            l2b = f2_add(l2b, f2_pack(p0, p1));
                         else
-                            l2 = f2_add(l2, f2_pack(p0, p1));
+                            l2a = f2_add(l2a, f2_pack(p0, p1));
                         w[i] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st16(tS + half * 32 + cc * 16, w);
+                    tmem_st16(tS + cc * 16, w);
                 }
-                l2 = f2_add(l2, lb2);
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
                     // O_X is stable (S_X(j) completing implies PV_X(j-1) completed) and PV_X(j)
-                    // cannot start before the arrive below: rescale this thread's half of the row
+                    // cannot start before the arrive below: rescale this thread's row
 #pragma unroll 1
                     for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[16];
-                        tmem_ld16(tO + cc * 16, o);
+                        uint32_t o[32];
+                        tmem_ld32p(tO + cc * 32, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
+                        for (int i = 0; i < 32; ++i)
                             o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st16(tO + cc * 16, o);
+                        tmem_st32(tO + cc * 32, o);
                     }
                 }
                 tmem_wait_st();
@@ -569,50 +640,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
             if (!ok)
                 break;
-            // ---- epilogue: O / l -> bf16 (this thread: half of the head dim)
-            if (!mbar_wait_warp(bar + (B_OF + x) * 8, titem & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            float la, lb;
-            f2_unpack(l2, la, lb);
-            const float l_half = la + lb;
-            // full row sum = both halves' partial sums.  A partner reads this slot right after
-            // the barrier, before its next step's barrier, so the slot is free again by the
-            // next item's epilogue.
-            lch[half * 128 + row] = l_half;
-            asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-            const float l_sum = l_half + lch[(half ^ 1) * 128 + row];
-            tc_fence_after();
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-            const bool store = row < g.rows;
-            const int t = gi.qs + gi.tok0 + x * TQ + row / G;
-            const int hq = gi.h * G + row % G;
-            __nv_bfloat16 *dst = p.out + ((int64_t)t * p.Hq + hq) * D + half * (D / 2);
-#pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[16];
-                tmem_ld16(tO + cc * 16, o);
-                tmem_wait_ld();
-                if (store) {
-#pragma unroll
-                    for (int i = 0; i < 16; i += 8) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
-                        v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-                        v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-                        v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(dst + cc * 16 + i) = v;
-                    }
-                }
-            }
-            // O_X may now be overwritten by the next item's first PV
-            tc_fence_before();
-            mbar_arrive(bar + (B_OE + x) * 8);
+            // row sum and reference max -> the epilogue warpgroup (slot by item parity; the
+            // epilogue reads it before it frees O_X, which this tile's next-but-one item waits for)
+            float la, lb, lc, ld;
+            f2_unpack(l2a, la, lb);
+            f2_unpack(l2b, lc, ld);
+            float *slot = lm + (titem & 1) * 256;
+            slot[row] = (la + lb) + (lc + ld);
+            slot[128 + row] = m_ref;
+            mbar_arrive(bar + (B_LF + x) * 8);
             ++titem;
-            if (store && p.lse && half == 0)
-                p.lse[(int64_t)t * p.Hq + hq] =
-                    l_sum > 0.f ? (m_ref * c + log2f(l_sum)) * 0.69314718055994531f : -CUDART_INF_F;
         }
         if (!ok && lane == 0)
             fail();
@@ -620,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -632,14 +669,24 @@ cudaError_t launch_prefill_t(const AttnParams &p, const CUtensorMap &tq, const C
 {
     constexpr int smem = PfCfg<D>::kSmem;
     static bool attr_done[64] = {};
+    static int regs_per_thread = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
         cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess)
             return e;
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, prefill_kernel<D>);
+        if (e != cudaSuccess)
+            return e;
+        regs_per_thread = fa.numRegs;
         attr_done[dev] = true;
     }
+    // The warpgroups' setmaxnreg budgets draw on the pool the CTA is launched with; a raise
+    // beyond it would wait forever, so never launch a build whose pool is smaller.
+    if (regs_per_thread >= 0 && regs_per_thread * kThreads < kRegSplit)
+        return cudaErrorInvalidConfiguration;
     // persistent: one CTA per SM, never more CTAs than the largest possible number of items
     const int64_t items = grid_tiles * p.Hkv;
     const unsigned grid = (unsigned)(items < num_sms ? items : num_sms);
