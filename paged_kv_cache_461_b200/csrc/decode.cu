@@ -32,6 +32,8 @@
 // an accumulator.
 #include <math_constants.h>
 
+#include <mutex>
+
 #include "merge.cuh"
 #include "pa_internal.cuh"
 #include "ptx.cuh"
@@ -479,15 +481,18 @@ cudaError_t launch_decode_t(const AttnParams &p, const CUtensorMap &tk, const CU
                             cudaStream_t s)
 {
     constexpr int smem = DecCfg<D, NT>::kSmem;
-    static bool attr_done[64] = {};
+    // the shared-memory attribute, once per device (host threads may call concurrently)
+    constexpr int kMaxDev = 64;
+    static std::once_flag once[kMaxDev];
+    static cudaError_t attr_err[kMaxDev];
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess)
-            return e;
-        attr_done[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [dev] {
+        attr_err[dev] = cudaFuncSetAttribute(decode_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err[dev] != cudaSuccess)
+        return attr_err[dev];
     const unsigned grid = (unsigned)(grid_units * p.Hkv); // (unit, kv head), heads of a unit adjacent
     decode_kernel<D, NT><<<grid, kDecWarps * 32, smem, s>>>(tk, tv, p);
     return cudaGetLastError();

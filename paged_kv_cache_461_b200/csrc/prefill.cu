@@ -53,6 +53,8 @@
 // never enters O.
 #include <math_constants.h>
 
+#include <mutex>
+
 #include "pa_internal.cuh"
 #include "tcgen05.cuh"
 
@@ -401,9 +403,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     break;
                 }
                 tc_fence_after();
+                // QK^T MMAs of this item still to issue: Q is released for the next item's load as soon
+                // as the last one is done, while this item's last PV MMAs and softmax still run
+                int s_left = nkt[0] + nkt[1];
+                auto s_issued = [&]() {
+                    if (--s_left == 0)
+                        umma_commit(bar + B_QE * 8);
+                };
                 for (int x = 0; x < 2; ++x)
-                    if (nkt[x] > 0)
+                    if (nkt[x] > 0) {
                         issue_s(x, gs);
+                        s_issued();
+                    }
                 umma_commit(bar + (B_KE + (gs & 1)) * 8); // K of step 0 consumed
                 for (int j = 0; ok && j < g.n_steps; ++j) {
                     const uint32_t gj = gs + j;
@@ -447,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                                 tc_fence_after();
                             }
                             issue_s(x, gj + 1);
+                            s_issued();
                         } else {
                             umma_commit(bar + (B_OF + x) * 8);
                         }
@@ -459,7 +471,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 }
                 if (!ok)
                     break;
-                umma_commit(bar + B_QE * 8); // Q of this item consumed
                 if (g.tail_fix)
                     ++nfix;
                 gs += g.n_steps;
@@ -668,24 +679,27 @@ cudaError_t launch_prefill_t(const AttnParams &p, const CUtensorMap &tq, const C
                              int64_t grid_tiles, int num_sms, cudaStream_t s)
 {
     constexpr int smem = PfCfg<D>::kSmem;
-    static bool attr_done[64] = {};
-    static int regs_per_thread = -1;
+    // once per device (host threads may call concurrently): the shared-memory attribute, and the
+    // registers per thread the kernel is launched with
+    constexpr int kMaxDev = 64;
+    static std::once_flag once[kMaxDev];
+    static cudaError_t attr_err[kMaxDev];
+    static int regs_per_thread[kMaxDev];
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess)
-            return e;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [dev] {
+        attr_err[dev] = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, prefill_kernel<D>);
-        if (e != cudaSuccess)
-            return e;
-        regs_per_thread = fa.numRegs;
-        attr_done[dev] = true;
-    }
+        if (attr_err[dev] == cudaSuccess)
+            attr_err[dev] = cudaFuncGetAttributes(&fa, prefill_kernel<D>);
+        regs_per_thread[dev] = attr_err[dev] == cudaSuccess ? fa.numRegs : 0;
+    });
+    if (attr_err[dev] != cudaSuccess)
+        return attr_err[dev];
     // The warpgroups' setmaxnreg budgets draw on the pool the CTA is launched with; a raise
     // beyond it would wait forever, so never launch a build whose pool is smaller.
-    if (regs_per_thread >= 0 && regs_per_thread * kThreads < kRegSplit)
+    if (regs_per_thread[dev] * kThreads < kRegSplit)
         return cudaErrorInvalidConfiguration;
     // persistent: one CTA per SM, never more CTAs than the largest possible number of items
     const int64_t items = grid_tiles * p.Hkv;
