@@ -23,9 +23,10 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller; only the
  *     pa_cache_desc_t / pa_attn_options_t structs are read from host memory,
  *     during the call (the prefix-cache functions are host-only, see there).
- *     The library never allocates device memory, frees or synchronises: work
- *     is enqueued on `stream` and the call returns at once (mixed steps also
- *     use one library-owned side stream, see pa_attention_mixed).
+ *     The library never allocates device memory, creates a stream or an
+ *     event, frees or synchronises: work is enqueued on `stream` (and, for a
+ *     mixed step, on the caller's side stream given in pa_attn_options_t) and
+ *     the call returns at once.
  *   - bf16 tensors are IEEE bfloat16 (2 bytes per element).
  *   - Host-side validation happens before anything is enqueued; a non-PA_OK
  *     status means nothing was enqueued, except PA_ERR_CUDA (a launch failed).
@@ -53,6 +54,8 @@ extern "C" {
 
 /* A cudaStream_t (the same handle type); NULL is the legacy default stream. */
 typedef struct CUstream_st *pa_stream_t;
+/* A cudaEvent_t (the same handle type). */
+typedef struct CUevent_st *pa_event_t;
 
 typedef enum pa_status {
     PA_OK = 0,
@@ -98,15 +101,33 @@ typedef struct pa_attn_options {
                                       instance under prefill/decode disaggregation); such a
                                       call never runs a decode grid beside prefill. */
     int32_t reserved[6];           /* must be zero */
+    /* How the two kernels of a step that holds both prefill-shaped and decode-shaped requests
+     * run.  The pages' V1 scheduler puts both kinds of work in one step (hn.213312.xyz section
+     * 一, "调度器"); prefill is bound by the tensor cores and decode by HBM, so they run best side
+     * by side.  side_stream: a second stream of the caller's, on the same device as `stream`,
+     * for the prefill kernel; fork_event / join_event: two events the call records and waits on
+     * to fork from `stream` and join back to it, so that the call stays one ordered unit on
+     * `stream` (and can be captured into a CUDA graph with `stream`).  All three NULL: the
+     * kernels run one after the other on `stream`.  Either all three or none (else
+     * INVALID_ARG); side_stream must differ from `stream`.  The caller owns them: the library
+     * creates no stream or event.  Calls that can be issued at the same time (other host
+     * threads, or other streams) need their own three. */
+    pa_stream_t side_stream;
+    pa_event_t fork_event;
+    pa_event_t join_event;
 } pa_attn_options_t;
 
 /* Bits of the device status word (uint32 at byte 0 of the workspace). */
-#define PA_DEVICE_BAD_SEQ 1u      /* a request had q_len < 0, seq_len < q_len, seq_len > max_seq_len or
-                                     query rows outside [0, num_tokens); it was skipped */
+#define PA_DEVICE_BAD_SEQ 1u      /* a request had q_len < 0, q_len > max_query_len, seq_len < q_len,
+                                     seq_len > max_seq_len or query rows outside [0, num_tokens); it was
+                                     skipped.  Also set when requests' query rows overlap (query_start_loc
+                                     decreasing somewhere) so far that their work does not fit the
+                                     workspace: the work that fits is done, the rest is dropped */
 #define PA_DEVICE_BAD_BLOCK 2u    /* a block id outside [0, num_blocks) was read (as zeros) */
 #define PA_DEVICE_WAIT_TIMEOUT 4u /* a kernel gave up waiting on a copy or a tensor-core result */
+#define PA_DEVICE_BAD_SLOT 8u     /* pa_kv_write_ex: a slot >= num_blocks*block_size was skipped */
 
-PA_API int32_t pa_abi_version(void); /* 2 */
+PA_API int32_t pa_abi_version(void); /* 3 */
 PA_API const char *pa_status_string(pa_status_t status);
 
 /*
@@ -131,6 +152,21 @@ PA_API pa_status_t pa_kv_write(const void *k_new, const void *v_new, int64_t new
                         const pa_cache_desc_t *cache, pa_stream_t stream);
 
 /*
+ * pa_kv_write_ex -- pa_kv_write that also reports slots outside the pool.
+ * (The pages' block manager hands out and takes back whole blocks on demand,
+ * shengyayun.com 关键实现细节 1, and the runner builds the slot mapping from
+ * those blocks while preparing inputs, hn.213312.xyz section 一; a slot past
+ * the pool therefore means corrupt metadata, which this call makes visible.)
+ * status: NULL, or a device uint32 (4-byte aligned, else INVALID_ARG) into
+ * which the kernel ORs PA_DEVICE_BAD_SLOT when a token's slot is >=
+ * num_blocks*block_size (that token is skipped as in pa_kv_write).  The call
+ * never clears it: the caller zeroes it before the calls it wants to check.
+ */
+PA_API pa_status_t pa_kv_write_ex(const void *k_new, const void *v_new, int64_t new_row_stride,
+                                  const int64_t *slot_mapping, int32_t num_tokens, void *k_cache, void *v_cache,
+                                  const pa_cache_desc_t *cache, uint32_t *status, pa_stream_t stream);
+
+/*
  * pa_build_slot_mapping -- the slot of every token of the step.
  * (hn.213312.xyz section 一, forward-pass paragraph: positions and the slot
  * mapping are prepared on the way into the forward pass.)
@@ -152,6 +188,11 @@ PA_API pa_status_t pa_build_slot_mapping(const int32_t *query_start_loc, const i
  * needs for these host-side bounds (0 on invalid arguments).  The value only
  * grows with each argument, so one workspace sized for the largest step of a
  * run serves every smaller step.
+ * (The pages' runner captures the forward pass in CUDA graphs when a worker
+ * starts, hn.213312.xyz section 一, and its KV tensors are allocated once up
+ * front; a step replayed from a graph cannot allocate, so the scratch a call
+ * needs -- work lists, split-KV partial states, the status word -- is sized
+ * here from host bounds alone and owned by the caller.)
  */
 PA_API size_t pa_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads,
                          const pa_cache_desc_t *cache, int32_t max_seq_len);
@@ -199,14 +240,16 @@ PA_API size_t pa_workspace_size_ex(int32_t num_seqs, int32_t num_tokens, int32_t
  * WORKSPACE_TOO_SMALL, CUDA.
  *
  * Concurrency inside a call: when a step can hold both prefill-shaped and
- * decode-shaped requests, the prefill kernel runs on a side stream of the
- * library, beside the decode kernel on `stream`, on an SM share the device
- * plan picks; `stream` waits for it before the call's work is complete (an
- * event fork/join, so the call is still one ordered unit on `stream` and can
- * be captured into a CUDA graph).  The side stream and its two events are
- * created on the first such call on a device and kept for the process; make
- * that first call outside stream capture.  This is the only resource the
- * library creates on its own.
+ * decode-shaped requests and options name a side stream and two events, the
+ * prefill kernel runs on the side stream beside the decode kernel on
+ * `stream`, on an SM share the device plan picks; `stream` waits for it
+ * before the call's work is complete (an event fork/join, so the call is
+ * still one ordered unit on `stream` and can be captured into a CUDA graph).
+ * Without them (and always for pa_attention_mixed) the prefill kernel takes
+ * every SM and the decode kernel runs after it on `stream`.  `stream` (and the
+ * side stream) must belong to the current device: every launch goes to the
+ * current device (the call does not query a stream's device, which is not
+ * allowed while the stream is being captured).
  */
 PA_API pa_status_t pa_attention_mixed(const void *q, int32_t num_q_heads, const void *k_cache,
                                const void *v_cache, const pa_cache_desc_t *cache,
@@ -241,8 +284,13 @@ PA_API pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, con
  *
  *  - The first call on a device looks up that device's copy of the array
  *    (cudaGetSymbolAddress) with the device current; make that first call
- *    before any stream capture on that device.  Later calls do no CUDA API
- *    work beyond the launches.
+ *    before any stream capture on that device.  As with every attention
+ *    entry point, the first launch of each kernel shape on a device (head
+ *    dim 64 or 128; decode-only, prefill-only or mixed) also sets that
+ *    kernel's shared-memory size attribute (cudaFuncSetAttribute) once.
+ *    Beyond those one-time calls a call does only its launches (and, for a
+ *    mixed step with the options' side stream, the event record / wait
+ *    pairs).
  *  - Bounds that need more than PA_NOALLOC_SCRATCH_BYTES of workspace
  *    (pa_workspace_size_ex(...) > PA_NOALLOC_SCRATCH_BYTES) are rejected with
  *    PA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued; a larger
@@ -252,6 +300,8 @@ PA_API pa_status_t pa_attention_mixed_ex(const void *q, int32_t num_q_heads, con
  *    it and give undefined results; calls ordered on one stream are safe.
  *    The array keeps the previous call's contents; each call re-initialises
  *    everything it reads (status word included) before reading it.
+ *  - The device status word (PA_DEVICE_* bits) sits in the array too; read
+ *    it with pa_noalloc_device_status after the call.
  *  - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
  */
 #define PA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
@@ -262,6 +312,18 @@ PA_API pa_status_t pa_attention_mixed_noalloc(const void *q, int32_t num_q_heads
                                               int32_t num_tokens, int32_t max_query_len, int32_t max_seq_len,
                                               float softmax_scale, void *out, float *lse,
                                               const pa_attn_options_t *options, pa_stream_t stream);
+
+/*
+ * pa_noalloc_device_status -- the device status word of the last
+ * pa_attention_mixed_noalloc call on the current device.  (No counterpart in
+ * the paper: the status word normally sits at byte 0 of the caller's
+ * workspace, and callers of the allocation-free entry point have none.)
+ * Enqueues one 4-byte copy on `stream` from the built-in array to status_out
+ * (host or device memory; a host pointer can be read once `stream` has
+ * synchronised).  Order it after the call on the same stream.  INVALID_ARG
+ * for a NULL status_out.
+ */
+PA_API pa_status_t pa_noalloc_device_status(uint32_t *status_out, pa_stream_t stream);
 
 /*
  * pa_merge_attn_states -- the split-KV reduce on its own.
@@ -394,6 +456,11 @@ PA_API int64_t pa_prefix_cache_size(pa_prefix_cache_t *cache); /* digests held, 
  * seq_len tokens of a cache, following its block table row (device int32
  * [ceil(seq_len/16)]).  out: bf16 [seq_len, num_kv_heads, head_dim].  A block
  * id outside the pool gives zero rows.
+ * (Token j of a request lives in block block_table[j / 16] at row j % 16 --
+ * the pages' fixed 16-token blocks handed out by the block manager,
+ * shengyayun.com 关键实现细节 1, indexed through the per-request block table,
+ * hn.213312.xyz section 一.  This copy lets tests check that index handling
+ * byte for byte against a plain walk of the table.)
  */
 PA_API pa_status_t pa_debug_gather_kv(const void *cache_ptr, const pa_cache_desc_t *cache, const int32_t *bt_row,
                                int32_t seq_len, void *out, pa_stream_t stream);

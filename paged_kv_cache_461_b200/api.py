@@ -12,6 +12,7 @@ from __future__ import annotations
 import ctypes
 import math
 import os
+import threading
 from typing import Optional
 
 import torch
@@ -25,13 +26,15 @@ STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3:
 DEVICE_BAD_SEQ = 1
 DEVICE_BAD_BLOCK = 2
 DEVICE_WAIT_TIMEOUT = 4
+DEVICE_BAD_SLOT = 8
 
 # every symbol include/pa.h declares
 EXPORTED = ("pa_abi_version", "pa_status_string", "pa_kv_write", "pa_build_slot_mapping", "pa_workspace_size",
             "pa_workspace_size_ex", "pa_attention_mixed", "pa_attention_mixed_ex", "pa_attention_mixed_noalloc",
             "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack", "pa_merge_attn_states", "pa_debug_gather_kv",
             "pa_prefix_block_hashes", "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_cache_insert",
-            "pa_prefix_cache_remove_block", "pa_prefix_cache_longest_hit", "pa_prefix_cache_size")
+            "pa_prefix_cache_remove_block", "pa_prefix_cache_longest_hit", "pa_prefix_cache_size", "pa_kv_write_ex",
+            "pa_noalloc_device_status")
 HASH_ALGOS = {"fnv1a64": 0, "sha256": 1}
 LAYOUT_HND = 0   # cache [num_blocks, num_kv_heads, 16, head_dim]
 LAYOUT_NHD = 1   # cache [num_blocks, 16, num_kv_heads, head_dim]
@@ -52,7 +55,8 @@ class CacheDesc(ctypes.Structure):
 
 class AttnOptions(ctypes.Structure):
     _fields_ = [("kv_split_tokens", ctypes.c_int32), ("decode_max_query_len", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("reserved", ctypes.c_int32 * 6), ("side_stream", ctypes.c_void_p), ("fork_event", ctypes.c_void_p),
+                ("join_event", ctypes.c_void_p)]
 
 
 _lib = None
@@ -70,6 +74,8 @@ def lib():
         L.pa_status_string.restype = ctypes.c_char_p
         L.pa_status_string.argtypes = [ctypes.c_int]
         L.pa_kv_write.argtypes = [_vp, _vp, _i64, _vp, _i32, _vp, _vp, ctypes.POINTER(CacheDesc), _vp]
+        L.pa_kv_write_ex.argtypes = [_vp, _vp, _i64, _vp, _i32, _vp, _vp, ctypes.POINTER(CacheDesc), _vp, _vp]
+        L.pa_noalloc_device_status.argtypes = [_vp, _vp]
         L.pa_build_slot_mapping.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp]
         L.pa_workspace_size.argtypes = [_i32, _i32, _i32, ctypes.POINTER(CacheDesc), _i32]
         L.pa_workspace_size.restype = _sz
@@ -102,7 +108,7 @@ def lib():
         L.pa_prefix_cache_longest_hit.restype = _i32
         L.pa_prefix_cache_size.argtypes = [_vp]
         L.pa_prefix_cache_size.restype = _i64
-        for name in ("pa_kv_write", "pa_build_slot_mapping", "pa_attention_mixed", "pa_attention_mixed_ex",
+        for name in ("pa_kv_write", "pa_kv_write_ex", "pa_noalloc_device_status", "pa_build_slot_mapping", "pa_attention_mixed", "pa_attention_mixed_ex",
                      "pa_attention_mixed_noalloc", "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack",
                      "pa_merge_attn_states", "pa_debug_gather_kv"):
             getattr(L, name).restype = ctypes.c_int
@@ -145,12 +151,54 @@ def cache_desc(k_cache: torch.Tensor, layout: str = "HND") -> CacheDesc:
     return CacheDesc(NB, Hkv, D, bs, _LAYOUTS[layout])
 
 
-def _opts(kv_split_tokens: int, decode_max_query_len: int = 0) -> Optional[AttnOptions]:
-    if not kv_split_tokens and not decode_max_query_len:
+# Side stream and fork/join events for running a mixed step's prefill kernel beside its decode kernel,
+# created with torch (the library creates none) and kept per (device, caller stream, host thread), so
+# that calls that may be issued at the same time never share them.
+_SIDE = {}
+_SIDE_LOCK = threading.Lock()
+
+
+def _side_resources(stream_ptr: int) -> tuple:
+    """(side stream, fork event, join event) for calls on the caller stream stream_ptr from this thread.
+    Created on first use: make the first call on a stream before capturing it into a CUDA graph."""
+    dev = torch.cuda.current_device()
+    key = (dev, stream_ptr, threading.get_ident())
+    with _SIDE_LOCK:
+        r = _SIDE.get(key)
+    if r is None:
+        side = torch.cuda.Stream(device=dev, priority=-100)  # maps to the device's highest priority
+        fork, join = torch.cuda.Event(), torch.cuda.Event()
+        fork.record(side)            # torch creates a CUDA event at its first record
+        join.record(side)
+        r = (side, fork, join)
+        with _SIDE_LOCK:
+            r = _SIDE.setdefault(key, r)
+    return r
+
+
+def _may_fork(num_q_heads: int, k_cache: torch.Tensor, layout: str, max_query_len: int,
+              decode_max_query_len: int) -> bool:
+    """Whether a call can hold both prefill-shaped and decode-shaped requests (only then does the library use a
+    side stream): a decode kernel exists and max_query_len reaches past the decode row limit."""
+    Hkv = k_cache.shape[1] if layout == "HND" else k_cache.shape[2]
+    G = max(1, num_q_heads // max(1, Hkv))
+    if decode_max_query_len == -1:
+        return False
+    cap = decode_max_query_len * G if decode_max_query_len > 0 else (8 if G <= 8 else 16)
+    return int(max_query_len) * G > cap
+
+
+def _opts(kv_split_tokens: int, decode_max_query_len: int = 0, stream_ptr: Optional[int] = None
+          ) -> Optional[AttnOptions]:
+    """Options of a call; with stream_ptr, also the binding's side stream and events for that caller stream."""
+    if not kv_split_tokens and not decode_max_query_len and stream_ptr is None:
         return None
     o = AttnOptions()
     o.kv_split_tokens = int(kv_split_tokens)
     o.decode_max_query_len = int(decode_max_query_len)
+    if stream_ptr is not None:
+        side, fork, join = _side_resources(stream_ptr)
+        o.side_stream, o.fork_event, o.join_event = side.cuda_stream, fork.cuda_event, join.cuda_event
     return o
 
 
@@ -222,15 +270,32 @@ def abi_version() -> int:
 
 
 def kv_write(k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor, k_cache: torch.Tensor,
-             v_cache: torch.Tensor, stream=None, layout: str = "HND") -> None:
-    """pa_kv_write: k_new/v_new [T, Hkv, D] (rows may be strided), slot_mapping int64 [T]."""
+             v_cache: torch.Tensor, stream=None, layout: str = "HND", status: Optional[torch.Tensor] = None) -> None:
+    """pa_kv_write: k_new/v_new [T, Hkv, D] (rows may be strided), slot_mapping int64 [T].
+    status (int32 [1] on the device, optional): pa_kv_write_ex ORs DEVICE_BAD_SLOT into it when a slot lies
+    outside the pool (the caller clears it)."""
     _need_caches(k_cache, v_cache)
     d = cache_desc(k_cache, layout)
     row_stride = _need_new_rows(k_new, v_new, d, k_cache.device)
     T = k_new.shape[0]
     _need(slot_mapping, torch.int64, "slot_mapping", shape=(T,), dense=True, device=k_cache.device)
-    _check(lib().pa_kv_write(_ptr(k_new), _ptr(v_new), row_stride, _ptr(slot_mapping), T, _ptr(k_cache),
-                             _ptr(v_cache), ctypes.byref(d), _stream(stream, k_cache.device)), "pa_kv_write")
+    if status is None:
+        _check(lib().pa_kv_write(_ptr(k_new), _ptr(v_new), row_stride, _ptr(slot_mapping), T, _ptr(k_cache),
+                                 _ptr(v_cache), ctypes.byref(d), _stream(stream, k_cache.device)), "pa_kv_write")
+        return
+    _need(status, torch.int32, "status", shape=(1,), dense=True, device=k_cache.device)
+    _check(lib().pa_kv_write_ex(_ptr(k_new), _ptr(v_new), row_stride, _ptr(slot_mapping), T, _ptr(k_cache),
+                                _ptr(v_cache), ctypes.byref(d), _ptr(status), _stream(stream, k_cache.device)),
+           "pa_kv_write_ex")
+
+
+def noalloc_device_status(stream=None) -> int:
+    """pa_noalloc_device_status: the PA_DEVICE_* bits of the last pa_attention_mixed_noalloc call on the current
+    device, read after the stream has finished the call."""
+    out = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = _stream(stream, out.device)
+    _check(lib().pa_noalloc_device_status(_ptr(out), st), "pa_noalloc_device_status")
+    return int(out.item())
 
 
 def build_slot_mapping(query_start_loc: torch.Tensor, seq_lens: torch.Tensor, block_table: torch.Tensor,
@@ -267,8 +332,10 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
                     softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                     lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                     kv_split_tokens: int = 0, decode_max_query_len: int = 0, stream=None,
-                    layout: str = "HND") -> torch.Tensor:
-    """pa_attention_mixed[_ex]: q [T, Hq, D] bf16 -> out [T, Hq, D] bf16 (lse [T, Hq] fp32 if given)."""
+                    layout: str = "HND", concurrent: bool = True) -> torch.Tensor:
+    """pa_attention_mixed[_ex]: q [T, Hq, D] bf16 -> out [T, Hq, D] bf16 (lse [T, Hq] fp32 if given).
+    concurrent: pass the binding's side stream and events for this caller stream, so that a step holding
+    both prefill and decode work runs the two kernels side by side (else one after the other)."""
     _need_q_out(q, out, lse)
     _need_caches(k_cache, v_cache, q.device)
     _need_meta(query_start_loc, seq_lens, block_table, q.device)
@@ -282,13 +349,15 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
         workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len, layout)
     _need(workspace, torch.uint8, "workspace", dense=True, device=q.device)
     d = cache_desc(k_cache, layout)
-    o = _opts(kv_split_tokens, decode_max_query_len)
+    st = _stream(stream, q.device)
+    fork = concurrent and _may_fork(Hq, k_cache, layout, max_query_len, decode_max_query_len)
+    o = _opts(kv_split_tokens, decode_max_query_len, (st.value or 0) if fork else None)
     _check(lib().pa_attention_mixed_ex(_ptr(q), Hq, _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
                                        _ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
                                        block_table.stride(0), R, T, int(max_query_len), int(max_seq_len),
                                        float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(),
-                                       ctypes.byref(o) if o else None, _stream(stream, q.device)), "pa_attention_mixed")
+                                       ctypes.byref(o) if o else None, st), "pa_attention_mixed")
     return out
 
 
@@ -296,7 +365,8 @@ def attention_mixed_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
                             query_start_loc: torch.Tensor, seq_lens: torch.Tensor, block_table: torch.Tensor,
                             max_query_len: int, max_seq_len: int, softmax_scale: Optional[float] = None,
                             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                            kv_split_tokens: int = 0, stream=None, layout: str = "HND") -> torch.Tensor:
+                            kv_split_tokens: int = 0, stream=None, layout: str = "HND",
+                            concurrent: bool = True) -> torch.Tensor:
     """pa_attention_mixed_noalloc: like attention_mixed but with the library's built-in scratch
     (for callers that cannot allocate a workspace; calls that overlap on the GPU race on it)."""
     _need_q_out(q, out, lse)
@@ -309,12 +379,14 @@ def attention_mixed_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
     if out is None:
         out = torch.empty_like(q)
     d = cache_desc(k_cache, layout)
-    o = _opts(kv_split_tokens)
+    st = _stream(stream, q.device)
+    fork = concurrent and _may_fork(Hq, k_cache, layout, max_query_len, 0)
+    o = _opts(kv_split_tokens, 0, (st.value or 0) if fork else None)
     _check(lib().pa_attention_mixed_noalloc(_ptr(q), Hq, _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
                                             _ptr(query_start_loc), _ptr(seq_lens), _ptr(block_table),
                                             block_table.stride(0), R, T, int(max_query_len), int(max_seq_len),
                                             float(softmax_scale), _ptr(out), _ptr(lse),
-                                            ctypes.byref(o) if o else None, _stream(stream, q.device)),
+                                            ctypes.byref(o) if o else None, st),
            "pa_attention_mixed_noalloc")
     return out
 

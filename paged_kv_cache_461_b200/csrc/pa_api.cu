@@ -3,6 +3,7 @@
 // sequence of one mixed step.  No function here allocates, frees or
 // synchronises; everything is enqueued on the caller's stream.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstring>
@@ -188,61 +189,36 @@ bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb)
     return na && nb && x < y + nb && y < x + na;
 }
 
+// SMs of the current device (looked up once per device)
 int device_sms()
 {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
+    constexpr int kMaxDev = 64;
+    static std::once_flag once[kMaxDev];
+    static int sms[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return 148;
+    std::call_once(once[dev], [dev] {
+        int n = 0;
+        sms[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
+    });
+    return sms[dev];
 }
 
 pa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
 
-// Per-device side stream and fork/join events for running the prefill kernel beside the
-// decode kernel of the same step.  Created on the first mixed call on a device and kept for
-// the life of the process.  The mutex orders the host-side record/wait pairs of concurrent
-// callers (the events are shared).
-struct SideStream {
-    cudaStream_t stream = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-    std::mutex mu;
-    bool ready = false;
+// An NVTX range around the launches of one entry point, so that a timeline (e.g. of a mixed step's
+// concurrent kernels) shows which call they belong to.  Costs a branch when no tool is attached.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
 };
-
-SideStream *side_stream()
-{
-    static SideStream table[64];
-    static std::mutex init_mu;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        return nullptr;
-    SideStream &ss = table[dev];
-    std::lock_guard<std::mutex> g(init_mu);
-    if (!ss.ready) {
-        if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
-            // release what was created, so a later call starts from nothing instead of leaking
-            if (ss.join)
-                cudaEventDestroy(ss.join);
-            if (ss.fork)
-                cudaEventDestroy(ss.fork);
-            if (ss.stream)
-                cudaStreamDestroy(ss.stream);
-            ss.stream = nullptr;
-            ss.fork = ss.join = nullptr;
-            return nullptr;
-        }
-        ss.ready = true;
-    }
-    return &ss;
-}
 
 } // namespace
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 2; }
+int32_t pa_abi_version(void) { return 3; }
 
 const char *pa_status_string(pa_status_t s)
 {
@@ -261,9 +237,9 @@ const char *pa_status_string(pa_status_t s)
     return "PA_ERR_UNKNOWN";
 }
 
-pa_status_t pa_kv_write(const void *k_new, const void *v_new, int64_t new_row_stride, const int64_t *slot_mapping,
-                        int32_t num_tokens, void *k_cache, void *v_cache, const pa_cache_desc_t *cache,
-                        pa_stream_t stream)
+pa_status_t pa_kv_write_ex(const void *k_new, const void *v_new, int64_t new_row_stride, const int64_t *slot_mapping,
+                           int32_t num_tokens, void *k_cache, void *v_cache, const pa_cache_desc_t *cache,
+                           uint32_t *status, pa_stream_t stream)
 {
     pa_status_t why;
     if (!cache_desc_ok(cache, &why))
@@ -274,9 +250,20 @@ pa_status_t pa_kv_write(const void *k_new, const void *v_new, int64_t new_row_st
         return PA_OK;
     if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache)
         return PA_ERR_INVALID_ARG;
+    if (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u))
+        return PA_ERR_INVALID_ARG;
+    NvtxRange r("pa_kv_write");
     return cuda_status(launch_kv_write(k_new, v_new, new_row_stride, slot_mapping, num_tokens, k_cache, v_cache,
                                        cache->num_blocks, cache->num_kv_heads, cache->head_dim,
-                                       cache->layout == PA_LAYOUT_NHD, reinterpret_cast<cudaStream_t>(stream)));
+                                       cache->layout == PA_LAYOUT_NHD, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+pa_status_t pa_kv_write(const void *k_new, const void *v_new, int64_t new_row_stride, const int64_t *slot_mapping,
+                        int32_t num_tokens, void *k_cache, void *v_cache, const pa_cache_desc_t *cache,
+                        pa_stream_t stream)
+{
+    return pa_kv_write_ex(k_new, v_new, new_row_stride, slot_mapping, num_tokens, k_cache, v_cache, cache, nullptr,
+                          stream);
 }
 
 pa_status_t pa_build_slot_mapping(const int32_t *query_start_loc, const int32_t *seq_lens, const int32_t *block_table,
@@ -289,6 +276,7 @@ pa_status_t pa_build_slot_mapping(const int32_t *query_start_loc, const int32_t 
         return PA_OK;
     if (!query_start_loc || !seq_lens || !block_table || !slot_mapping || bt_stride == 0)
         return PA_ERR_INVALID_ARG;
+    NvtxRange r("pa_build_slot_mapping");
     return cuda_status(launch_slot_mapping(query_start_loc, seq_lens, block_table, bt_stride, num_seqs, num_tokens,
                                            slot_mapping, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -331,6 +319,13 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     if (!make_plan(num_seqs, num_tokens, num_q_heads, cache, max_seq_len, options, P, &why))
         return why;
     if (max_query_len < 0 || bt_stride < 0 || !std::isfinite(softmax_scale))
+        return PA_ERR_INVALID_ARG;
+    // the caller's side stream and fork/join events for running prefill beside decode: all or none
+    cudaStream_t side = options ? reinterpret_cast<cudaStream_t>(options->side_stream) : nullptr;
+    cudaEvent_t ev_fork = options ? reinterpret_cast<cudaEvent_t>(options->fork_event) : nullptr;
+    cudaEvent_t ev_join = options ? reinterpret_cast<cudaEvent_t>(options->join_event) : nullptr;
+    if ((side != nullptr) != (ev_fork != nullptr) || (side != nullptr) != (ev_join != nullptr) ||
+        (side != nullptr && (side == reinterpret_cast<cudaStream_t>(stream) || ev_fork == ev_join)))
         return PA_ERR_INVALID_ARG;
     if ((int64_t)bt_stride * kBlockSize < (int64_t)max_seq_len)
         return PA_ERR_INVALID_ARG;
@@ -390,6 +385,9 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     p.num_seqs = num_seqs;
     p.num_tokens = num_tokens;
     p.max_seq_len = max_seq_len;
+    p.max_query_len = max_query_len;
+    p.max_dec_units = P.max_dec_units;
+    p.max_pf_tiles = P.max_pf_tiles;
     p.Hq = num_q_heads;
     p.Hkv = Hkv;
     p.G = P.G;
@@ -421,35 +419,31 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     if (prefill && !get_map(q, 3, D, (uint64_t)num_q_heads, (uint64_t)num_tokens, (uint32_t)P.G,
                             (uint32_t)(kPrefillRows / P.G), &tq))
         return PA_ERR_CUDA;
-    // A mixed step forks after the plan: prefill (persistent, on the plan's share of the SMs, at
-    // the highest priority) on the side stream, decode (with its split merge) on the caller's
-    // stream, which then waits for prefill.  The two kernels never touch the same output rows.
-    SideStream *ss = (prefill && P.NT > 0) ? side_stream() : nullptr;
-    if (prefill && P.NT > 0 && !ss)
-        return PA_ERR_CUDA;
+    // A mixed step with a side stream forks after the plan: prefill (persistent, on the plan's share
+    // of the SMs, at the highest priority) on the side stream, decode (with its split merge) on the
+    // caller's stream, which then waits for prefill.  The two kernels never touch the same output
+    // rows.  Without a side stream prefill takes every SM and decode follows it on `stream`.
+    const bool fork = prefill && P.NT > 0 && side != nullptr;
+    p.pf_all_sms = fork ? 0 : 1;
+    NvtxRange range(fw ? "pa_attention_decode_fused" : "pa_attention_mixed");
     cudaError_t e = launch_plan(p, s);
     if (e != cudaSuccess)
         return PA_ERR_CUDA;
-    std::unique_lock<std::mutex> fork_lock;
-    if (ss) {
-        fork_lock = std::unique_lock<std::mutex>(ss->mu);
-        if (cudaEventRecord(ss->fork, s) != cudaSuccess || cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
-            return PA_ERR_CUDA;
-    }
+    if (fork && (cudaEventRecord(ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess))
+        return PA_ERR_CUDA;
     if (prefill) {
-        e = launch_prefill(p, tq, tk, tv, P.max_pf_tiles, p.num_sms, ss ? ss->stream : s);
+        e = launch_prefill(p, tq, tk, tv, P.max_pf_tiles, p.num_sms, fork ? side : s);
         if (e != cudaSuccess)
             return PA_ERR_CUDA;
     }
-    if (ss && cudaEventRecord(ss->join, ss->stream) != cudaSuccess)
+    if (fork && cudaEventRecord(ev_join, side) != cudaSuccess)
         return PA_ERR_CUDA;
     if (P.NT > 0) {
         e = launch_decode(p, tk, tv, P.NT, P.max_dec_units, s);
         if (e != cudaSuccess)
             return PA_ERR_CUDA;
-
     }
-    if (ss && cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
+    if (fork && cudaStreamWaitEvent(s, ev_join, 0) != cudaSuccess)
         return PA_ERR_CUDA;
     return PA_OK;
 }
@@ -505,8 +499,9 @@ pa_status_t pa_kv_pack(const void *k_cache, const void *v_cache, const pa_cache_
         return PA_ERR_INVALID_ARG;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(staging) || !aligned16(block_ids))
         return PA_ERR_UNSUPPORTED;
+    NvtxRange r("pa_kv_pack");
     return cuda_status(launch_kv_pack(k_cache, v_cache, cache->num_blocks, block_elems, block_ids, num_ids, staging,
-                                      device_sms(), reinterpret_cast<cudaStream_t>(stream)));
+                                      device_sms(), nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 pa_status_t pa_kv_unpack(const void *staging, const int32_t *block_ids, int32_t num_ids, void *k_cache,
@@ -529,8 +524,9 @@ pa_status_t pa_kv_unpack(const void *staging, const int32_t *block_ids, int32_t 
         return PA_ERR_INVALID_ARG;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(staging) || !aligned16(block_ids))
         return PA_ERR_UNSUPPORTED;
+    NvtxRange r("pa_kv_unpack");
     return cuda_status(launch_kv_unpack(staging, block_ids, num_ids, k_cache, v_cache, cache->num_blocks, block_elems,
-                                        device_sms(), reinterpret_cast<cudaStream_t>(stream)));
+                                        device_sms(), nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 pa_status_t pa_attention_mixed(const void *q, int32_t num_q_heads, const void *k_cache, const void *v_cache,
@@ -558,6 +554,7 @@ pa_status_t pa_merge_attn_states(const float *part_out, const float *part_lse, c
         return PA_ERR_INVALID_ARG;
     if (!aligned16(part_out) || (reinterpret_cast<uintptr_t>(out) & 7u))
         return PA_ERR_UNSUPPORTED;
+    NvtxRange r("pa_merge_attn_states");
     return cuda_status(launch_merge_states(part_out, part_lse, parts_per_row, num_rows, num_heads, num_parts, head_dim,
                                            out, lse_out, reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -56,6 +56,9 @@ struct AttnParams {
     int num_seqs;
     int num_tokens;
     int max_seq_len;
+    int max_query_len;          // host bound of q_len; a request above it is skipped (PA_DEVICE_BAD_SEQ)
+    int64_t max_dec_units;      // room of the decode work list in the workspace
+    int64_t max_pf_tiles;       // room of the prefill work list in the workspace
     int Hq, Hkv, G, D;
     float scale_log2;           // softmax_scale * log2(e)
     WsHeader *hdr;
@@ -67,6 +70,7 @@ struct AttnParams {
     int split_tokens, max_splits, QD, dec_rows_cap;
     int nhd;                    // cache layout PA_LAYOUT_NHD (else HND)
     int num_sms;                // SMs of the device (the plan splits them between prefill and decode)
+    int pf_all_sms;             // 1: prefill runs alone (every SM); 0: beside decode on the plan's share
     // fused KV write (pa_attention_decode_fused); k_new == nullptr otherwise
     const uint16_t *k_new, *v_new;
     int64_t new_row_stride;     // elements
@@ -76,11 +80,12 @@ struct AttnParams {
 // launchers (return cudaGetLastError() of the launch)
 cudaError_t launch_kv_write(const void *k_new, const void *v_new, int64_t row_stride, const int64_t *slots,
                             int num_tokens, void *k_cache, void *v_cache, int64_t num_blocks, int Hkv, int D,
-                            int nhd, cudaStream_t s);
+                            int nhd, uint32_t *status, cudaStream_t s);
 cudaError_t launch_kv_pack(const void *k_cache, const void *v_cache, int64_t num_blocks, int64_t block_elems,
-                           const int32_t *ids, int num_ids, void *staging, int num_sms, cudaStream_t s);
+                           const int32_t *ids, int num_ids, void *staging, int num_sms, uint32_t *status,
+                           cudaStream_t s);
 cudaError_t launch_kv_unpack(const void *staging, const int32_t *ids, int num_ids, void *k_cache, void *v_cache,
-                             int64_t num_blocks, int64_t block_elems, int num_sms, cudaStream_t s);
+                             int64_t num_blocks, int64_t block_elems, int num_sms, uint32_t *status, cudaStream_t s);
 cudaError_t launch_slot_mapping(const int32_t *qsl, const int32_t *seq_lens, const int32_t *bt, int bt_stride,
                                 int num_seqs, int num_tokens, int64_t *slots, cudaStream_t s);
 cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D, int nhd, const int32_t *bt_row,

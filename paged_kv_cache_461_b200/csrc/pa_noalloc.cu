@@ -62,3 +62,17 @@ extern "C" PA_API pa_status_t pa_attention_mixed_noalloc(const void *q, int32_t 
                                  bt_stride, num_seqs, num_tokens, max_query_len, max_seq_len, softmax_scale, out, lse,
                                  scratch, PA_NOALLOC_SCRATCH_BYTES, options, stream);
 }
+
+extern "C" PA_API pa_status_t pa_noalloc_device_status(uint32_t *status_out, pa_stream_t stream)
+{
+    if (!status_out)
+        return PA_ERR_INVALID_ARG;
+    void *scratch = scratch_for_current_device();
+    if (!scratch)
+        return PA_ERR_CUDA;
+    // the status word is the first field of the workspace header, at byte 0
+    return cudaMemcpyAsync(status_out, scratch, sizeof(uint32_t), cudaMemcpyDefault,
+                           reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
+}

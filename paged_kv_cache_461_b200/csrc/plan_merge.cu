@@ -154,7 +154,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
         const int qs = p.qsl[r], qe = p.qsl[r + 1];
         q_len = qe - qs;
         const int L = p.seq_lens[r];
-        const bool bad = qs < 0 || qe > p.num_tokens || q_len < 0 || L < q_len || L > p.max_seq_len;
+        const bool bad = qs < 0 || qe > p.num_tokens || q_len < 0 || q_len > p.max_query_len || L < q_len ||
+                         L > p.max_seq_len;
         if (bad) {
             atomicOr(&hdr->status, PA_DEVICE_BAD_SEQ);
             q_len = 0;
@@ -189,7 +190,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
         int ed, ep, er, td, tp, tr;
         cta_excl_scan3(n_dec, n_pf, red, ed, ep, er, td, tp, tr);
         for (int s = 0; s < n_dec; ++s)
-            p.dec_units[carry_dec + ed + s] = make_int2(r, s);
+            if (carry_dec + ed + s < p.max_dec_units)
+                p.dec_units[carry_dec + ed + s] = make_int2(r, s);
         if (red)
             for (int h = 0; h < p.Hkv; ++h)
                 p.split_arrivals[(int64_t)r * p.Hkv + h] = 0u; // counted by the decode kernel
@@ -220,7 +222,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
                 classify(r, n_dec, n_pf, red, ctx, q_len);
             for (int k = 0; k < n_pf; ++k) {
                 const int pos = atomicAdd(&hist[min(pair_cost(ctx, q_len, k, tq), n_buckets - 1)], 1);
-                p.pf_tiles[pos] = make_int2(r, k);
+                if (pos < p.max_pf_tiles) // only overlapping query rows can exceed the list (flagged below)
+                    p.pf_tiles[pos] = make_int2(r, k);
             }
         }
     }
@@ -242,10 +245,15 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
     }
     const float dec_bytes = (float)dec_tokens * (float)(p.Hkv * p.D * 4); // K + V, bf16
     const float pf_flops = (float)pf_pairs * (float)(4 * p.Hq * p.D);
-    const int pf_ctas = choose_pf_ctas(pf_flops, dec_bytes, p.num_sms, carry_pf * p.Hkv);
+    const int pf_ctas = p.pf_all_sms ? max(1, min(p.num_sms, carry_pf * p.Hkv))
+                                     : choose_pf_ctas(pf_flops, dec_bytes, p.num_sms, carry_pf * p.Hkv);
     if (threadIdx.x == 0) {
-        hdr->n_dec_units = (uint32_t)carry_dec;
-        hdr->n_pf_tiles = (uint32_t)carry_pf;
+        // Requests whose query rows overlap (a query_start_loc that decreases somewhere) can ask for more
+        // work items than the host-sized lists hold: keep what fits, flag the step.
+        if (carry_dec > p.max_dec_units || carry_pf > p.max_pf_tiles)
+            atomicOr(&hdr->status, PA_DEVICE_BAD_SEQ);
+        hdr->n_dec_units = (uint32_t)min((int64_t)carry_dec, p.max_dec_units);
+        hdr->n_pf_tiles = (uint32_t)min((int64_t)carry_pf, p.max_pf_tiles);
         hdr->n_reduce = (uint32_t)carry_red;
 #ifdef PA_FORCE_PF_CTAS
         hdr->pf_ctas = (uint32_t)min(PA_FORCE_PF_CTAS, p.num_sms);

@@ -47,7 +47,7 @@ def test_library_exports_nothing_else(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.pa_abi_version() == 2
+    assert L.pa_abi_version() == 3
     for code, name in api.STATUS_NAMES.items():
         assert L.pa_status_string(code).decode() == name
 
@@ -191,6 +191,34 @@ def _fused(L, **kw):
                                        ctypes.byref(a["desc"]), a["qsl"], a["sl"], a["bt"], a["bts"], a["R"], a["T"],
                                        a["mq"], a["ms"], ctypes.c_float(a["scale"]), a["out"], a["lse"], a["ws"],
                                        a["wsb"], a["opt"], None)
+
+
+def _mixed(L, **kw):
+    a = dict(q=FAKE, hq=32, k=FAKE + (1 << 31), v=FAKE + (1 << 31) + (1 << 29), desc=_desc(), qsl=FAKE, sl=FAKE,
+             bt=FAKE, bts=64, R=4, T=4, mq=1, ms=1000, scale=0.088, out=FAKE + (1 << 30), lse=None,
+             ws=FAKE + (1 << 32), wsb=1 << 30, opt=None, stream=None)
+    a.update(kw)
+    return L.pa_attention_mixed_ex(a["q"], a["hq"], a["k"], a["v"], ctypes.byref(a["desc"]), a["qsl"], a["sl"],
+                                   a["bt"], a["bts"], a["R"], a["T"], a["mq"], a["ms"], ctypes.c_float(a["scale"]),
+                                   a["out"], a["lse"], a["ws"], a["wsb"], a["opt"], a["stream"])
+
+
+def test_side_stream_and_events_come_all_or_none(L):
+    # the caller's side stream and fork/join events for a mixed step: all three or none, and the side
+    # stream differs from the call's stream; the library never creates them itself
+    def opts(side=None, fork=None, join=None):
+        o = api.AttnOptions()
+        o.side_stream, o.fork_event, o.join_event = side, fork, join
+        return ctypes.byref(o)
+    assert _mixed(L, opt=opts(side=FAKE)) == 1
+    assert _mixed(L, opt=opts(side=FAKE, fork=FAKE + 64)) == 1
+    assert _mixed(L, opt=opts(fork=FAKE + 64, join=FAKE + 128)) == 1
+    assert _mixed(L, opt=opts(side=FAKE, fork=FAKE + 64, join=FAKE + 64)) == 1       # one event for both
+    assert _mixed(L, opt=opts(side=FAKE, fork=FAKE + 64, join=FAKE + 128), stream=FAKE) == 1   # side == stream
+    # all three given (or none): passes these checks and stops only at the (absent) driver
+    assert _mixed(L, opt=opts(side=FAKE, fork=FAKE + 64, join=FAKE + 128)) in (0, 4)
+    assert _mixed(L, opt=opts()) in (0, 4)
+    assert ctypes.sizeof(api.AttnOptions) == 32 + 3 * ctypes.sizeof(ctypes.c_void_p)
 
 
 def test_fused_decode_host_validation(L):

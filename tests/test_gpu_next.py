@@ -228,12 +228,14 @@ def test_step_replays_from_a_cuda_graph_bit_identically(kind):
     lay = _layout("graph", ctx, q, 32, 8, 128, seed=17)
     st = DevStep(lay, W.make_values_numpy(lay))
     st.write()
-    out_e, lse_e = st.attend()                       # eager call first (creates the side stream)
+    cap = torch.cuda.Stream()
+    with torch.cuda.stream(cap):                     # eager call on the capture stream first: the binding
+        out_e, lse_e = st.attend()                   # makes that stream's side stream and events here
     torch.cuda.synchronize()
     out_g = torch.full_like(out_e, float("nan"))
     lse_g = torch.full_like(lse_e, float("nan"))
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    with torch.cuda.graph(g, stream=cap):
         api.attention_mixed(st.q, st.k_cache, st.v_cache, st.qsl, st.seq_lens, st.bt, lay.max_query_len,
                             lay.max_seq_len, out=out_g, lse=lse_g, workspace=st.workspace)
     for _ in range(2):

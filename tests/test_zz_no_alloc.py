@@ -81,3 +81,20 @@ def test_noalloc_rejects_bounds_beyond_its_scratch():
                                               1 << 40, 8192, 4096, 4096, 1, 131072, ctypes.c_float(0.08),
                                               (1 << 40) + (1 << 36), None, None, None)
     assert rc == 3  # PA_ERR_WORKSPACE_TOO_SMALL, nothing enqueued
+
+
+def test_noalloc_status_word_is_readable():
+    # the allocation-free call's device status word lives in the built-in scratch; the accessor copies
+    # it out.  A block id outside the pool is read as zeros and flagged; the next clean call clears it.
+    build.build()
+    lay, vals = _batch(33)
+    st = DevStep(lay, vals)
+    st.write()
+    good_bt = st.bt
+    st.bt = good_bt.clone()
+    st.bt[0, 0] = lay.num_blocks + 77
+    _noalloc_call(st, 0)
+    assert api.noalloc_device_status() & api.DEVICE_BAD_BLOCK
+    st.bt = good_bt
+    _noalloc_call(st, 0)
+    assert api.noalloc_device_status() == 0
