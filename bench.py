@@ -175,6 +175,12 @@ def whole_job_value(bytes_per_rank: float, ms_per_step_local: float, ws: int) ->
     return ws * bytes_per_rank / (ms * 1e-3) / 1e9, ms
 
 
+def job_config(lay, n_gpus: int) -> dict:
+    """The `config` object of both arms: the workload and how the job is laid out, nothing arm-specific."""
+    return {**lay.describe(), "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single device",
+            "step": "KV write of the step's new rows + attention over the whole batch"}
+
+
 # --------------------------------------------------------------------------- our arm
 
 class Step:
@@ -263,6 +269,61 @@ def _attention_only_ms(st: Step, steps: int):
         evs.append((a, b))
     torch.cuda.synchronize()
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def _window(fn, seconds: float = 0.3, min_steps: int = 50):
+    """Back-to-back steps for about `seconds` (at least min_steps), each bracketed by its own CUDA events on the
+    launching stream: (median ms, mean ms, steps, host seconds)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(5):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    n = max(min_steps, int(seconds * 1e3 / max(a.elapsed_time(b) / 5, 1e-3)))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    h0 = time.monotonic()
+    for e0, e1 in evs:
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    h1 = time.monotonic()
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    return statistics.median(ms), statistics.mean(ms), n, h1 - h0
+
+
+def _kv_write_alone(st: "Step", peaks: dict, launches: int = 100):
+    """pa_kv_write of the mixed step's 8192 new tokens on its own: each launch timed by its own events, with a
+    256 MB buffer read between launches so that neither the new rows nor their cache slots are still in
+    L2 (126 MB) -- read, not written, so that L2 holds no dirty lines that the write would have to evict
+    first.  Algorithmic bytes: the new K and V rows read once and written once."""
+    import torch
+    lay = st.lay
+    valid = int((lay.slot_mapping >= 0).sum())
+    moved = 2 * 2 * valid * lay.num_kv_heads * lay.head_dim * 2   # (K, V) x (read, write) x bf16
+    flush = torch.zeros(64 << 20, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        st.kv_write()
+    ms = []
+    for _ in range(launches):
+        flush.sum()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        st.kv_write()
+        b.record(stream)
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    del flush
+    med = statistics.median(ms)
+    gbs = moved / (med * 1e-3) / 1e9
+    return {"ms_per_launch": med, "ms_mean": statistics.mean(ms), "launches": launches, "tokens": valid,
+            "bytes_read_plus_written": moved, "value": gbs, "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+            "peak": peaks["hbm_gbs"], "l2": "256 MB read between launches (cold, clean L2)",
+            "workload": lay.name}, launches
 
 
 def _prefill_only(st: Step, steps: int, warmup: int):
@@ -594,18 +655,22 @@ def _cpu_model() -> str:
 
 
 def reference_arm(args, ws, rank):
-    """The reference arm: the fp64 oracle, as it stands, on this machine's host cores.  Rank 0 alone
-    runs it (other ranks exit without work).  Each step is one oracle pass of the same step our arm
-    times (KV write, then attention) over a bounded sample of the workload: its first 8 requests."""
+    """The reference arm: the fp64 oracle, as it stands, on this machine's host cores, over the whole workload
+    (every request).  Rank 0 alone runs it (other ranks exit without work).  Each timed step is one oracle
+    attention pass over the batch; the oracle's KV write (a pure function that returns copies of both pools)
+    runs once before the steps and is timed on its own, outside the steps."""
     if rank != 0:
         return
     import oracle
     from paged_kv_cache_461_b200 import workloads as W
     full = W.workload_layout(args.workload)
-    sub, vals = _oracle_sample(args.workload, 8)
+    n_req = full.num_seqs if args.reference_requests <= 0 else min(args.reference_requests, full.num_seqs)
+    sub, vals = _oracle_sample(args.workload, n_req)
+    t0 = time.perf_counter()
+    kc, vc = oracle.kv_write(vals.k_new, vals.v_new, sub.slot_mapping, vals.k_cache, vals.v_cache)
+    write_s = time.perf_counter() - t0
 
     def step():
-        kc, vc = oracle.kv_write(vals.k_new, vals.v_new, sub.slot_mapping, vals.k_cache, vals.v_cache)
         oracle.attention_for(sub, kc, vc, vals.q)
 
     t0 = time.perf_counter()
@@ -623,14 +688,16 @@ def reference_arm(args, ws, rank):
     dt = statistics.mean(t_steps)
     v = sub.kv_bytes() / dt / 1e9
     cores = oracle.num_cores()
-    sample = f"first {sub.num_seqs} of the {full.num_seqs} requests of {args.workload}, each step one oracle pass " \
-             f"(KV write + attention, fp64, {cores} threads)"
+    which = f"all {sub.num_seqs}" if sub.num_seqs == full.num_seqs else f"the first {sub.num_seqs} of {full.num_seqs}"
+    sample = f"{which} requests of {args.workload} ({sub.kv_bytes() / 1e9:.3f} GB of KV), each step one " \
+             f"oracle attention pass (fp64, {cores} threads); the oracle's KV write timed once outside the steps"
     line = {"metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus, "steps": len(t_steps),
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {**full.describe(), "parallelism": "host cores (oracle)", "sample_requests": sub.num_seqs,
-                       "step": "oracle.kv_write + oracle.attention"},
-            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "config": job_config(full, args.gpus),
+            "oracle_kv_write_ms": write_s * 1e3,
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
+                             "cpu_model": _cpu_model()},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -678,6 +745,39 @@ def profile_case(kind: str, launches: int):
                       "pool_bytes": 2 * v.k_cache.numel() * 2}))
 
 
+def _summary(line: dict) -> dict:
+    """The headline numbers of every part of the line in one short object, printed last."""
+    r = lambda x, n=4: None if x is None else round(float(x), n)
+    out = {"headline_gbs": r(line["value"], 1), "headline_frac": r(line["roofline"]["frac"]),
+           "headline_ms_median": r(line["window"]["ms_per_step_median"], 5)}
+    m = line.get("mixed_step")
+    if m:
+        out.update({"mixed_ms": r(m["ms_per_step"], 5), "mixed_tok_s": r(m["value"], 0),
+                    "prefill_tflops": r(m["prefill_roofline"]["achieved"], 1),
+                    "prefill_frac": r(m["prefill_roofline"]["frac"])})
+    w = line.get("kv_write")
+    if w:
+        out.update({"kv_write_gbs": r(w["value"], 1), "kv_write_frac": r(w["frac"])})
+    f = line.get("follow_on")
+    if f:
+        for k, short in (("fused_kv_write_decode", "fused"), ("nhd_decode", "nhd"), ("kv_pack", "pack"),
+                         ("kv_unpack", "unpack"), ("spec_verify_k3", "spec_k3")):
+            if k in f:
+                out[f"{short}_gbs"] = r(f[k]["value"], 1)
+                out[f"{short}_frac"] = r(f[k]["frac"])
+    o = line.get("other_workloads")
+    if o:
+        for k, short in (("long_context_decode", "long_ctx"), ("prefix_sharing", "prefix")):
+            if k in o:
+                out[f"{short}_gbs"] = r(o[k]["value"], 1)
+                out[f"{short}_frac"] = r(o[k]["frac"])
+    if "e2e" in line:
+        out["e2e_gbs"] = r(line["e2e"]["value"], 1)
+    if "cpu_baseline" in line:
+        out["cpu_oracle_gbs"] = r(line["cpu_baseline"]["value"], 3)
+    return out
+
+
 # --------------------------------------------------------------------------- main
 
 def main():
@@ -688,6 +788,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-requests", type=int, default=0,
+                    help="reference arm: time only the first N requests (0 = the whole workload)")
     ap.add_argument("--no-extras", action="store_true", help="headline only (no mixed step, e2e, prefill)")
     ap.add_argument("--profile-case", choices=["decode", "spec", "prefill"],
                     help="run a small case of one kernel for an ncu capture and exit")
@@ -716,7 +818,11 @@ def main():
     sampler = ClockSampler(local)
     win = []
     ms_total = _time_region(st.step, args.steps, args.warmup, ws, window=win)
-    clocks = sampler.stop(*win)
+    # the same step back to back for about 0.3 s right after the timed region, each step on its own events:
+    # the median per-step time, and enough clock samples to see the clocks the timed steps ran at
+    w_med, w_mean, w_n, w_s = _window(st.step)
+    clocks = sampler.stop(win[0], time.monotonic())
+    clocks["note"] = "samples over the timed region and the 0.3 s window of the same step right after it"
     value, ms_step = whole_job_value(st.kv_bytes, ms_total / args.steps, ws)
 
     # dominant kernel roofline: the attention launches (plan + decode with its split merge), events on their stream
@@ -731,11 +837,12 @@ def main():
 
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {**st.lay.describe(), "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                       "l2": f"inputs larger than L2 ({st.kv_bytes / 1e9:.2f} GB KV read per step), no flush",
-                       "step": "pa_kv_write + pa_attention_mixed"},
-            "roofline": roofline, "gpu_launches": st.launches_per_step * args.steps, "clocks": clocks}
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": job_config(st.lay, ws),
+            "l2": f"inputs larger than L2 ({st.kv_bytes / 1e9:.2f} GB of KV read per step), no flush",
+            "calls_per_step": "pa_kv_write + pa_attention_mixed",
+            "window": {"ms_per_step_median": w_med, "ms_per_step_mean": w_mean, "steps": w_n, "seconds": w_s,
+                       "value_median": ws * st.kv_bytes / (w_med * 1e-3) / 1e9},
+            "roofline": roofline, "gpu_launches": st.launches_per_step * (args.steps + w_n + 5), "clocks": clocks}
 
     if not args.no_extras:
         # every rank runs its replica end to end; the job's step time is the slowest rank's
@@ -772,10 +879,13 @@ def main():
                                  "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                                  "clocks": pf_clocks}}
         line["gpu_launches"] += mx.launches_per_step * mk
+        line["kv_write"], n_w = _kv_write_alone(mx, peaks)
+        line["gpu_launches"] += n_w + 3
 
     if ws == 1 and not args.no_cpu_baseline:
         # the oracle on this machine's host cores, at N = 1 only (a multi-GPU run would hold every GPU meanwhile)
         line["cpu_baseline"] = cpu_oracle_run(args.workload)
+    line["summary"] = _summary(line)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:

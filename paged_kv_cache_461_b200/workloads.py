@@ -34,10 +34,16 @@ BF16_QNAN = 0x7FC0
 # ----------------------------------------------------------------------------
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 values to bf16 (nearest even) and return the uint16 bit patterns."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    bias = ((u >> np.uint64(16)) & np.uint64(1)) + np.uint64(0x7FFF)
-    return ((u + bias) >> np.uint64(16)).astype(np.uint16)
+    """Round fp32 values to bf16 (nearest even) and return the uint16 bit patterns.
+    Works through the array in pieces so that the 64-bit temporaries stay small for multi-GB pools."""
+    flat = np.ascontiguousarray(x, dtype=np.float32).reshape(-1).view(np.uint32)
+    out = np.empty(flat.shape, dtype=np.uint16)
+    step = 1 << 23
+    for s in range(0, flat.size, step):
+        u = flat[s:s + step].astype(np.uint64)
+        bias = ((u >> np.uint64(16)) & np.uint64(1)) + np.uint64(0x7FFF)
+        out[s:s + step] = ((u + bias) >> np.uint64(16)).astype(np.uint16)
+    return out.reshape(np.shape(x))
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

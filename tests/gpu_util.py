@@ -4,20 +4,26 @@ measure the difference.  Marshalling only -- no attention arithmetic here.
 
 Parity gate (from the stated target: max-abs 2e-2, max-rel 1e-2 on bf16
 outputs computed with fp32 accumulation):
-  * max_abs  = max over all elements |gpu - oracle|                 <= 2e-2
+  * |gpu - oracle| <= 2e-2 + half a bf16 ulp of |oracle|, per element (below)
   * max_rel  = max over (token, head) rows of
                max_d |gpu - oracle| / max(max_d |oracle|, 1e-2)     <= 1e-2
     i.e. the error of each head's output vector relative to that vector's
     magnitude (a per-element ratio is meaningless for outputs near zero);
   * lse: max |gpu - oracle| <= 1e-3.
-Where outputs exceed 2.5 in magnitude (stress inputs with V ~ N(3, 1)) bf16's
-own spacing is coarser than 2e-2 (one ulp is 2^-5 in [4, 8)), so the abs gate
-becomes two bf16 half-ulps of the largest output, 2^-7 * max|oracle|; it is
-never looser than that and never tighter than 2e-2.
+The abs gate is applied per element as 2e-2 plus half a bf16 ulp of that
+element's exact value: the output itself is rounded to bf16, which alone can
+move an element by half an ulp (2^-6 for |O| in [4, 8), more than 2e-2 would
+leave for the arithmetic), and an element below 2 gets at most 2e-2 + 2^-8.
+The per-element relative error |gpu - oracle| / max(|oracle|, 1e-2) is also
+measured and reported (max_rel_elem); it is not gated, since near-zero outputs
+make it a ratio of rounding noise to nothing.  With PA_PARITY_LOG set to a
+file path, every checked case appends one JSON line with these statistics.
 """
 from __future__ import annotations
 
+import json
 import math
+import os
 
 import numpy as np
 import torch
@@ -128,27 +134,43 @@ def oracle_for_step(layout: W.StepLayout, vals: W.StepValues, scale=None, token_
     return oracle.attention_for(layout, kc, vc, vals.q, scale=scale, token_list=token_list)
 
 
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers at |x| (8 significant bits): 2^(e - 9) for |x| = m * 2^e, m in [0.5, 1)."""
+    _, e = np.frexp(np.abs(x))
+    return np.where(x == 0, 0.0, np.ldexp(1.0, e - 9))
+
+
 def errors(gpu_out: torch.Tensor, ref: np.ndarray, rows=None) -> dict:
     g = bf16_to_f64(gpu_out)
     if rows is not None:
         g = g[rows]
     d = np.abs(g - ref)
     if d.size == 0:
-        return {"max_abs": 0.0, "max_rel": 0.0, "nan": False}
+        return {"max_abs": 0.0, "max_rel": 0.0, "max_rel_elem": 0.0, "abs_over_gate": 0.0, "nan": False}
     nan = bool(np.isnan(g).any())
     row_err = d.max(axis=-1)
     row_mag = np.maximum(np.abs(ref).max(axis=-1), 1e-2)
     rel = row_err / row_mag
+    rel_elem = d / np.maximum(np.abs(ref), 1e-2)
+    gate = ATOL + bf16_half_ulp(ref)
     i = np.unravel_index(int(np.nanargmax(d)), d.shape)
-    return {"max_abs": float(np.nanmax(d)), "max_rel": float(np.nanmax(rel)), "argmax": tuple(int(x) for x in i),
-            "nan": nan}
+    return {"max_abs": float(np.nanmax(d)), "max_rel": float(np.nanmax(rel)),
+            "max_rel_elem": float(np.nanmax(rel_elem)), "abs_over_gate": float(np.nanmax(d / gate)),
+            "argmax": tuple(int(x) for x in i), "nan": nan}
+
+
+def _log(what: str, e: dict):
+    path = os.environ.get("PA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": what, **{k: v for k, v in e.items() if k != "argmax"}}) + "\n")
 
 
 def assert_parity(gpu_out, ref, gpu_lse=None, ref_lse=None, rows=None, what=""):
     e = errors(gpu_out, ref, rows)
+    _log(what, e)
     assert not e["nan"], f"{what}: NaN in GPU output"
-    atol = max(ATOL, 2.0 ** -7 * float(np.abs(ref).max()) if np.size(ref) else 0.0)
-    assert e["max_abs"] <= atol, f"{what}: max_abs {e} (gate {atol})"
+    assert e["abs_over_gate"] <= 1.0, f"{what}: |err| above 2e-2 + half a bf16 ulp somewhere: {e}"
     assert e["max_rel"] <= RTOL, f"{what}: max_rel {e}"
     if gpu_lse is not None and ref_lse is not None:
         gl = gpu_lse.cpu().numpy().astype(np.float64)

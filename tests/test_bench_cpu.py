@@ -17,8 +17,10 @@ def _bench(*args, env=None):
 
 
 def test_reference_arm_prints_one_contract_line():
+    # the default arm times every request of the workload; 8 keep this test short
     import bench
-    r = _bench("--impl", "reference", "--steps", "3", "--warmup", "3")
+    from paged_kv_cache_461_b200 import workloads as W
+    r = _bench("--impl", "reference", "--steps", "3", "--warmup", "3", "--reference-requests", "8")
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -29,9 +31,11 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["metric"] == bench.METRIC
     assert d["value"] > 0 and d["unit"] == "GB/s" and d["higher_is_better"] is True
     assert d["steps"] == 3 and d["warmup"] == 3 and d["n_gpus"] == 1
-    assert d["config"]["workload"] == bench.HEADLINE and d["config"]["sample_requests"] == 8
+    # the same config object as our arm's line (the whole workload), so the two lines compare
+    assert d["config"] == bench.job_config(W.workload_layout(bench.HEADLINE), 1)
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert cb["sample"].startswith("the first 8 of 256 requests") and d["oracle_kv_write_ms"] > 0
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
