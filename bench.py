@@ -296,34 +296,54 @@ def _window(fn, seconds: float = 0.3, min_steps: int = 50):
 
 
 def _kv_write_alone(st: "Step", peaks: dict, launches: int = 100):
-    """pa_kv_write of the mixed step's 8192 new tokens on its own: each launch timed by its own events, with a
-    256 MB buffer read between launches so that neither the new rows nor their cache slots are still in
-    L2 (126 MB) -- read, not written, so that L2 holds no dirty lines that the write would have to evict
-    first.  Algorithmic bytes: the new K and V rows read once and written once."""
+    """pa_kv_write of the mixed step's 8192 new tokens on its own, back to back: launches cycle through four
+    input sets (the step's own new rows and slots, and three more 8192-token sets whose slots come from the
+    same workload drawn with other seeds), so the rows read and the slots written (4 x 64 MB) exceed L2
+    (126 MB) and every launch goes to HBM.  CUDA events around the whole loop; per-launch time = total / launches.
+    Also the median of single launches, each after a 256 MB read that leaves L2 cold and clean.  The extra sets
+    overwrite cache slots of the step's pool, so this runs after everything else that uses that pool.
+    Algorithmic bytes: the new K and V rows read once and written once."""
     import torch
-    lay = st.lay
+    from paged_kv_cache_461_b200 import workloads as W
+    lay, v = st.lay, st.vals
+    sets = [(v.k_new, v.v_new, st.slots)]
+    for seed in (13, 23, 33):
+        other = W.workload_layout(lay.name, seed)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed)
+        kn = torch.randn(v.k_new.shape, generator=g, device="cuda").to(torch.bfloat16)
+        vn = torch.randn(v.v_new.shape, generator=g, device="cuda").to(torch.bfloat16)
+        sets.append((kn, vn, torch.from_numpy(other.slot_mapping).cuda()))
     valid = int((lay.slot_mapping >= 0).sum())
     moved = 2 * 2 * valid * lay.num_kv_heads * lay.head_dim * 2   # (K, V) x (read, write) x bf16
-    flush = torch.zeros(64 << 20, dtype=torch.float32, device="cuda")
+    run = lambda i: st.api.kv_write(sets[i % 4][0], sets[i % 4][1], sets[i % 4][2], v.k_cache, v.v_cache)
+    for i in range(8):
+        run(i)
+    torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    for _ in range(3):
-        st.kv_write()
-    ms = []
-    for _ in range(launches):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(launches):
+        run(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / launches
+    flush = torch.zeros(64 << 20, dtype=torch.float32, device="cuda")
+    cold = []
+    for i in range(20):
         flush.sum()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        st.kv_write()
-        b.record(stream)
-        b.synchronize()
-        ms.append(a.elapsed_time(b))
-    del flush
-    med = statistics.median(ms)
-    gbs = moved / (med * 1e-3) / 1e9
-    return {"ms_per_launch": med, "ms_mean": statistics.mean(ms), "launches": launches, "tokens": valid,
-            "bytes_read_plus_written": moved, "value": gbs, "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-            "peak": peaks["hbm_gbs"], "l2": "256 MB read between launches (cold, clean L2)",
-            "workload": lay.name}, launches
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run(i)
+        e1.record(stream)
+        e1.synchronize()
+        cold.append(e0.elapsed_time(e1))
+    del flush, sets
+    gbs = moved / (ms * 1e-3) / 1e9
+    return {"ms_per_launch": ms, "launches": launches, "tokens": valid, "bytes_read_plus_written": moved,
+            "value": gbs, "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+            "l2": "back to back over 4 input sets of 64 MB each (more than L2)",
+            "ms_single_cold_launch": statistics.median(cold), "workload": lay.name}, launches + 28
 
 
 def _prefill_only(st: Step, steps: int, warmup: int):
@@ -709,13 +729,38 @@ def profile_case(kind: str, launches: int):
     """A reduced copy of a workload for ncu (same shapes, fewer requests, pool sized to fit):
     decode: the first 64 requests of the Llama-3-8B-shaped decode batch (~0.6 GB of KV, above L2);
     spec: the same 64 requests verifying 3 drafted tokens each (q_len 4, decode_max_query_len 4);
-    prefill: the prefill chunks of the mixed 8192-token step alone.
+    prefill: the prefill chunks of the mixed 8192-token step alone;
+    kvwrite: pa_kv_write of the mixed step's 8192 new tokens (pool sized to its requests, ~2 GB per cache);
+    pack: pa_kv_pack of every block of the headline batch's first 64 requests.
     Runs 1 warm-up launch of pa_attention_mixed and then `launches` more."""
     import torch
 
     from paged_kv_cache_461_b200 import api, build
     from paged_kv_cache_461_b200 import workloads as W
     build.build()
+    if kind in ("kvwrite", "pack"):
+        # the mixed step's 8192-token KV write / whole-block pack of the headline batch's first 64 requests
+        # (a pool sized to the requests' blocks, so the capture holds a few GB at most)
+        lay = W.workload_layout(MIXED if kind == "kvwrite" else HEADLINE)
+        idx = np.arange(64) if kind == "pack" else np.arange(lay.num_seqs)
+        lay = W.build_layout(f"{lay.name}_{kind}_case", lay.ctx_lens[idx], lay.q_lens[idx],
+                             num_q_heads=lay.num_q_heads, num_kv_heads=lay.num_kv_heads, head_dim=lay.head_dim,
+                             seed=lay.seed)
+        v = W.make_values_torch(lay, "cuda")
+        slots = torch.from_numpy(lay.slot_mapping).cuda()
+        nblk = (lay.seq_lens + 15) // 16
+        ids = torch.from_numpy(np.concatenate([lay.block_table[r, :n] for r, n in enumerate(nblk)]).astype(np.int32)).cuda()
+        staging = torch.empty((len(ids), 2, lay.num_kv_heads * 16 * lay.head_dim), dtype=torch.bfloat16, device="cuda")
+        for _ in range(1 + launches):
+            if kind == "kvwrite":
+                api.kv_write(v.k_new, v.v_new, slots, v.k_cache, v.v_cache)
+            else:
+                api.kv_pack(v.k_cache, v.v_cache, ids, staging)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": kind, **lay.describe(), "blocks": len(ids),
+                          "bytes_moved": 2 * staging.numel() * 2 if kind == "pack" else
+                          4 * int((lay.slot_mapping >= 0).sum()) * lay.num_kv_heads * lay.head_dim * 2}))
+        return
     full = W.workload_layout(MIXED if kind == "prefill" else HEADLINE)
     if kind in ("decode", "spec"):
         idx = np.arange(64)
@@ -791,7 +836,7 @@ def main():
     ap.add_argument("--reference-requests", type=int, default=0,
                     help="reference arm: time only the first N requests (0 = the whole workload)")
     ap.add_argument("--no-extras", action="store_true", help="headline only (no mixed step, e2e, prefill)")
-    ap.add_argument("--profile-case", choices=["decode", "spec", "prefill"],
+    ap.add_argument("--profile-case", choices=["decode", "spec", "prefill", "kvwrite", "pack"],
                     help="run a small case of one kernel for an ncu capture and exit")
     args = ap.parse_args()
     if args.profile_case:
@@ -818,15 +863,17 @@ def main():
     sampler = ClockSampler(local)
     win = []
     ms_total = _time_region(st.step, args.steps, args.warmup, ws, window=win)
-    # the same step back to back for about 0.3 s right after the timed region, each step on its own events:
-    # the median per-step time, and enough clock samples to see the clocks the timed steps ran at
+    # dominant kernel roofline: the attention launches (plan + decode with its split merge), events on their
+    # stream, right after the timed steps (before the long window below warms the GPU into its power cap)
+    att_ms = _attention_only_ms(st, max(20, min(args.steps, 200)))
+    # the same step back to back for about 0.3 s, each step on its own events: the median per-step time, and
+    # enough clock samples to see the clocks the timed steps ran at
     w_med, w_mean, w_n, w_s = _window(st.step)
     clocks = sampler.stop(win[0], time.monotonic())
-    clocks["note"] = "samples over the timed region and the 0.3 s window of the same step right after it"
+    clocks["note"] = "samples over the timed region, the attention-only launches and the 0.3 s window of the " \
+                     "same step after them"
     value, ms_step = whole_job_value(st.kv_bytes, ms_total / args.steps, ws)
 
-    # dominant kernel roofline: the attention launches (plan + decode with its split merge), events on their stream
-    att_ms = _attention_only_ms(st, max(20, min(args.steps, 200)))
     achieved = st.kv_bytes / (att_ms * 1e-3) / 1e9
     traffic, _ = _traffic("decode_llama3_8b_decode", ["decode.cu", "ptx.cuh", "pa_internal.cuh"])
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -880,7 +927,7 @@ def main():
                                  "clocks": pf_clocks}}
         line["gpu_launches"] += mx.launches_per_step * mk
         line["kv_write"], n_w = _kv_write_alone(mx, peaks)
-        line["gpu_launches"] += n_w + 3
+        line["gpu_launches"] += n_w
 
     if ws == 1 and not args.no_cpu_baseline:
         # the oracle on this machine's host cores, at N = 1 only (a multi-GPU run would hold every GPU meanwhile)

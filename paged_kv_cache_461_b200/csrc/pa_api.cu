@@ -501,7 +501,7 @@ pa_status_t pa_kv_pack(const void *k_cache, const void *v_cache, const pa_cache_
         return PA_ERR_UNSUPPORTED;
     NvtxRange r("pa_kv_pack");
     return cuda_status(launch_kv_pack(k_cache, v_cache, cache->num_blocks, block_elems, block_ids, num_ids, staging,
-                                      device_sms(), nullptr, reinterpret_cast<cudaStream_t>(stream)));
+                                      device_sms(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 pa_status_t pa_kv_unpack(const void *staging, const int32_t *block_ids, int32_t num_ids, void *k_cache,
@@ -526,7 +526,7 @@ pa_status_t pa_kv_unpack(const void *staging, const int32_t *block_ids, int32_t 
         return PA_ERR_UNSUPPORTED;
     NvtxRange r("pa_kv_unpack");
     return cuda_status(launch_kv_unpack(staging, block_ids, num_ids, k_cache, v_cache, cache->num_blocks, block_elems,
-                                        device_sms(), nullptr, reinterpret_cast<cudaStream_t>(stream)));
+                                        device_sms(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 pa_status_t pa_attention_mixed(const void *q, int32_t num_q_heads, const void *k_cache, const void *v_cache,

@@ -82,10 +82,9 @@ cudaError_t launch_kv_write(const void *k_new, const void *v_new, int64_t row_st
                             int num_tokens, void *k_cache, void *v_cache, int64_t num_blocks, int Hkv, int D,
                             int nhd, uint32_t *status, cudaStream_t s);
 cudaError_t launch_kv_pack(const void *k_cache, const void *v_cache, int64_t num_blocks, int64_t block_elems,
-                           const int32_t *ids, int num_ids, void *staging, int num_sms, uint32_t *status,
-                           cudaStream_t s);
+                           const int32_t *ids, int num_ids, void *staging, int num_sms, cudaStream_t s);
 cudaError_t launch_kv_unpack(const void *staging, const int32_t *ids, int num_ids, void *k_cache, void *v_cache,
-                             int64_t num_blocks, int64_t block_elems, int num_sms, uint32_t *status, cudaStream_t s);
+                             int64_t num_blocks, int64_t block_elems, int num_sms, cudaStream_t s);
 cudaError_t launch_slot_mapping(const int32_t *qsl, const int32_t *seq_lens, const int32_t *bt, int bt_stride,
                                 int num_seqs, int num_tokens, int64_t *slots, cudaStream_t s);
 cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D, int nhd, const int32_t *bt_row,
