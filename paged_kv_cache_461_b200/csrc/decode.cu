@@ -90,9 +90,10 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
     const int L = p.seq_lens[r];
     const int ctx = L - q_len;
     const int rows = q_len * p.G;
-    const int k_begin = split * p.split_tokens;
-    const int k_end = min(L, k_begin + p.split_tokens);
-    const int n_splits = (L + p.split_tokens - 1) / p.split_tokens;
+    const int split_tokens = (int)p.hdr->split_tokens; // the plan's choice for this step
+    const int k_begin = split * split_tokens;
+    const int k_end = min(L, k_begin + split_tokens);
+    const int n_splits = (L + split_tokens - 1) / split_tokens;
     const int nb = (k_end - k_begin + kBlockSize - 1) / kBlockSize;
     const int blk0 = k_begin / kBlockSize;
 

@@ -400,6 +400,7 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     p.part_o = reinterpret_cast<float *>(ws + P.off_part_o);
     p.part_lse = reinterpret_cast<float *>(ws + P.off_part_lse);
     p.split_tokens = P.split_tokens;
+    p.auto_split = (options && options->kv_split_tokens) ? 0 : 1;
     p.max_splits = P.max_splits;
     p.QD = P.QD;
     p.dec_rows_cap = P.dec_rows_cap;

@@ -24,7 +24,8 @@ struct WsHeader {
     uint32_t n_pf_tiles;  // (request, q-tile) prefill work items
     uint32_t n_reduce;    // decode requests with more than one split (merged by their last split CTA)
     uint32_t pf_ctas;     // persistent prefill CTAs that take work; the others leave their SM to decode
-    uint32_t pad[59];
+    uint32_t split_tokens; // keys per split-KV partition of this step's decode requests
+    uint32_t pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -68,6 +69,7 @@ struct AttnParams {
     float *part_o;              // [num_seqs*QD*Hq*max_splits, D]
     float *part_lse;            // [num_seqs*QD*Hq*max_splits]
     int split_tokens, max_splits, QD, dec_rows_cap;
+    int auto_split;             // 1: the plan may take 2x or 4x split_tokens (the caller left the split to the library)
     int nhd;                    // cache layout PA_LAYOUT_NHD (else HND)
     int num_sms;                // SMs of the device (the plan splits them between prefill and decode)
     int pf_all_sms;             // 1: prefill runs alone (every SM); 0: beside decode on the plan's share

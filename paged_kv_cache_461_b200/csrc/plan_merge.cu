@@ -78,6 +78,7 @@ __device__ __forceinline__ void cta_excl_scan3(int a, int b, int c, int &ea, int
 //   decode   ~65 GB/s per SM (two CTAs, ~190 KB of loads in flight per SM, so latency
 //            bound when confined to part of the GPU), at most the HBM rate.
 constexpr float kPfFlopsPerSm = 6.2e12f;
+constexpr int kDecCtasPerSm = 12; // decode CTAs per SM below which the plan keeps the shorter split
 constexpr float kDecBytesPerSm = 65e9f;
 constexpr float kDecBytesMax = 6.35e12f;
 
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
         hist[i] = 0;
     __syncthreads();
     const int tq = kPrefillRows / p.G;
+    // n_dec: splits of a decode request at the host's split size (0 for every other request)
     auto classify = [&](int r, int &n_dec, int &n_pf, int &red, int &ctx, int &q_len) {
         n_dec = n_pf = red = 0;
         ctx = q_len = 0;
@@ -171,32 +173,64 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
             n_pf = (q_len * p.G + kPrefillRowsPerCta - 1) / kPrefillRowsPerCta;
         }
     };
-    // pass 1: decode units in request order, split-arrival counters zeroed; histogram of prefill pair costs
-    int carry_dec = 0, carry_pf = 0, carry_red = 0;
-    int kept_pf = 0, kept_ctx = 0, kept_q = 0; // this thread's request when one pass covers them all
+    // pass 1: classification, histogram of prefill pair costs, and the decode units the step would
+    // have at two and four times the host's split size
+    int carry_pf = 0, carry_u2 = 0, carry_u4 = 0;
+    int kept_pf = 0, kept_ctx = 0, kept_q = 0, kept_L = 0; // this thread's request when one pass covers them all
+    const int s2 = 2 * p.split_tokens, s4 = 4 * p.split_tokens;
     for (int base = 0; base < p.num_seqs; base += blockDim.x) {
         const int r = base + threadIdx.x;
         int n_dec, n_pf, red, ctx, q_len;
         classify(r, n_dec, n_pf, red, ctx, q_len);
+        const int L = n_dec ? ctx + q_len : 0; // keys of a decode request
         kept_pf = n_pf;
         kept_ctx = ctx;
         kept_q = q_len;
+        kept_L = L;
         for (int k = 0; k < n_pf; ++k)
             atomicAdd(&hist[min(pair_cost(ctx, q_len, k, tq), n_buckets - 1)], 1);
         if (n_dec)
-            my_dec_tokens += (unsigned long long)(ctx + q_len);
+            my_dec_tokens += (unsigned long long)L;
         if (n_pf)
             my_pf_pairs += (unsigned long long)q_len * ctx + (unsigned long long)q_len * (q_len + 1) / 2;
-        int ed, ep, er, td, tp, tr;
-        cta_excl_scan3(n_dec, n_pf, red, ed, ep, er, td, tp, tr);
-        for (int s = 0; s < n_dec; ++s)
-            if (carry_dec + ed + s < p.max_dec_units)
-                p.dec_units[carry_dec + ed + s] = make_int2(r, s);
+        int e0, e1, e2, tp, t2, t4;
+        cta_excl_scan3(n_pf, (L + s2 - 1) / s2, (L + s4 - 1) / s4, e0, e1, e2, tp, t2, t4);
+        carry_pf += tp;
+        carry_u2 += t2;
+        carry_u4 += t4;
+    }
+    // Split size of this step.  A decode CTA has a fixed cost (barrier setup, the first loads in
+    // flight, the partial-state write and merge), so fewer, longer splits read HBM faster as long as
+    // there are still about a dozen CTAs per SM to balance.  The caller's explicit split is kept.
+    int split = p.split_tokens;
+    if (p.auto_split) {
+        const int64_t want = (int64_t)kDecCtasPerSm * p.num_sms;
+        if ((int64_t)carry_u4 * p.Hkv >= want)
+            split = s4;
+        else if ((int64_t)carry_u2 * p.Hkv >= want)
+            split = s2;
+    }
+    // pass 1b: decode units in request order at that split size, split-arrival counters zeroed
+    int carry_dec = 0, carry_red = 0;
+    for (int base = 0; base < p.num_seqs; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        int L = kept_L;
+        if (p.num_seqs > (int)blockDim.x) {
+            int n_dec, n_pf, red, ctx, q_len;
+            classify(r, n_dec, n_pf, red, ctx, q_len);
+            L = n_dec ? ctx + q_len : 0;
+        }
+        const int n_dec = (L + split - 1) / split;
+        const int red = n_dec > 1 ? 1 : 0;
+        int ed, er, e2, td, tr, t2;
+        cta_excl_scan3(n_dec, red, 0, ed, er, e2, td, tr, t2);
+        for (int u = 0; u < n_dec; ++u)
+            if (carry_dec + ed + u < p.max_dec_units)
+                p.dec_units[carry_dec + ed + u] = make_int2(r, u);
         if (red)
             for (int h = 0; h < p.Hkv; ++h)
                 p.split_arrivals[(int64_t)r * p.Hkv + h] = 0u; // counted by the decode kernel
         carry_dec += td;
-        carry_pf += tp;
         carry_red += tr;
     }
     __syncthreads();
@@ -255,6 +289,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
         hdr->n_dec_units = (uint32_t)min((int64_t)carry_dec, p.max_dec_units);
         hdr->n_pf_tiles = (uint32_t)min((int64_t)carry_pf, p.max_pf_tiles);
         hdr->n_reduce = (uint32_t)carry_red;
+        hdr->split_tokens = (uint32_t)split;
 #ifdef PA_FORCE_PF_CTAS
         hdr->pf_ctas = (uint32_t)min(PA_FORCE_PF_CTAS, p.num_sms);
 #else

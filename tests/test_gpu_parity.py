@@ -423,6 +423,45 @@ def test_split_and_unsplit_decode_agree():
     assert (la - lb).abs().max().item() <= 1e-3
 
 
+def _expected_split(lay, sms):
+    """The plan's per-step split rule restated on the host: 4x or 2x the 1024-key default while the
+    step's decode requests still give at least 12 split CTAs per SM, else the default."""
+    L = (lay.ctx_lens + lay.q_lens).astype(np.int64)
+    dec = (lay.q_lens > 0) & (lay.q_lens * (lay.num_q_heads // lay.num_kv_heads) <= 8)
+    want = 12 * sms
+    for split in (4096, 2048):
+        if int(np.sum((L[dec] + split - 1) // split)) * lay.num_kv_heads >= want:
+            return split
+    return 1024
+
+
+@pytest.mark.parametrize("n_req,lo,hi", [(240, 100, 1000), (120, 2100, 3000), (12, 500, 9000)])
+def test_plan_picks_the_split_size_per_step(n_req, lo, hi):
+    # with the split left to the library the plan takes longer splits when the step has decode work
+    # enough to keep every SM busy with them; the result is bit-identical to asking for that split
+    rng = np.random.default_rng(n_req)
+    ctx = rng.integers(lo, hi, size=n_req)
+    lay = _layout("autosplit", ctx, np.ones(n_req, np.int32), 32, 8, 64, seed=n_req)
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    out, lse = st.attend()
+    torch.cuda.synchronize()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    split = st.workspace[20:24].view(torch.int32).item()
+    assert split == _expected_split(lay, sms), split
+    ref, ref_lse, _ = oracle_for_step(lay, vals)
+    assert_parity(out, ref, lse, ref_lse, what=f"auto split {split}")
+    out_x, lse_x = st.attend(kv_split_tokens=split)
+    torch.cuda.synchronize()
+    assert st.workspace[20:24].view(torch.int32).item() == split
+    assert torch.equal(out, out_x) and torch.equal(lse, lse_x)
+    if split != 1024:  # an explicit split is used as given
+        st.attend(kv_split_tokens=1024)
+        torch.cuda.synchronize()
+        assert st.workspace[20:24].view(torch.int32).item() == 1024
+
+
 # ----------------------------------------------------------------------------- device-side checks
 
 def test_bad_metadata_sets_status_and_never_faults():
