@@ -338,12 +338,31 @@ def _kv_write_alone(st: "Step", peaks: dict, launches: int = 100):
         e1.record(stream)
         e1.synchronize()
         cold.append(e0.elapsed_time(e1))
-    del flush, sets
+    # size-matched reference: a plain device copy (torch's copy kernel) of the same K and V rows into four
+    # rotating contiguous destinations, back to back -- what moving these bytes costs without the scatter
+    dst = [(torch.empty_like(v.k_new), torch.empty_like(v.v_new)) for _ in range(4)]
+    copy = lambda i: (dst[i % 4][0].copy_(sets[i % 4][0]), dst[i % 4][1].copy_(sets[i % 4][1]))
+    for i in range(8):
+        copy(i)
+    torch.cuda.synchronize()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for i in range(launches):
+        copy(i)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    copy_ms = c0.elapsed_time(c1) / launches
+    del flush, sets, dst
     gbs = moved / (ms * 1e-3) / 1e9
     return {"ms_per_launch": ms, "launches": launches, "tokens": valid, "bytes_read_plus_written": moved,
             "value": gbs, "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
             "l2": "back to back over 4 input sets of 64 MB each (more than L2)",
-            "ms_single_cold_launch": statistics.median(cold), "workload": lay.name}, launches + 28
+            "ms_single_cold_launch": statistics.median(cold),
+            "same_bytes_device_copy": {"ms": copy_ms, "value": moved / (copy_ms * 1e-3) / 1e9, "unit": "GB/s",
+                                       "frac_of_it": copy_ms / ms,
+                                       "what": "torch copy_ of the same K and V rows into 4 rotating contiguous "
+                                               "buffers, back to back (two copy kernels per set)"},
+            "workload": lay.name}, launches + 28
 
 
 def _prefill_only(st: Step, steps: int, warmup: int):
@@ -802,7 +821,8 @@ def _summary(line: dict) -> dict:
                     "prefill_frac": r(m["prefill_roofline"]["frac"])})
     w = line.get("kv_write")
     if w:
-        out.update({"kv_write_gbs": r(w["value"], 1), "kv_write_frac": r(w["frac"])})
+        out.update({"kv_write_gbs": r(w["value"], 1), "kv_write_frac": r(w["frac"]),
+                    "kv_write_vs_same_bytes_copy": r(w["same_bytes_device_copy"]["frac_of_it"])})
     f = line.get("follow_on")
     if f:
         for k, short in (("fused_kv_write_decode", "fused"), ("nhd_decode", "nhd"), ("kv_pack", "pack"),

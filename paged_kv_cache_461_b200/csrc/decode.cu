@@ -43,11 +43,12 @@ namespace {
 
 constexpr int kDecWarps = 4;
 
-// Ring depth per warp: 3 blocks for 8 packed rows (2 CTAs per SM), 2 for 16 rows, where
-// each block takes twice the work and 3 CTAs per SM (12 warps) hide more of it.
+// Ring depth per warp: 2 blocks, so 3 CTAs (12 warps, 24 blocks = 192 KB of loads in flight)
+// fit per SM; the extra warps hide the per-block MMA and softmax latency better than a third
+// stage per warp with 2 CTAs per SM (same bytes in flight).
 template <int D, int NT>
 struct DecCfg {
-    static constexpr int kStages = NT == 1 ? 3 : 2;
+    static constexpr int kStages = 2;
     static constexpr int kHalves = D / 64;
     static constexpr int kBox = 16 * 64 * 2;           // one TMA box: 16 rows x 64 bf16
     static constexpr int kTile = kHalves * kBox;       // one (block, kv head) of K or V

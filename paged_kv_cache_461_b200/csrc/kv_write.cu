@@ -37,6 +37,24 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const uint16_t *__restric
     for (int64_t t = (int64_t)blockIdx.x * warps_per_cta + (threadIdx.x >> 5); t < num_tokens;
          t += (int64_t)gridDim.x * warps_per_cta) {
         const int64_t slot = slots[t];
+        const uint16_t *ks = k_new + t * row_stride;
+        const uint16_t *vs = v_new + t * row_stride;
+        // Up to four vectors of K and four of V per lane: the first group is loaded before the
+        // slot is known (the token's rows are always readable), so the two loads overlap.
+        Vec kv[4], vv[4];
+        auto load = [&](int i0) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * 32;
+                if (i < vec_per_tok) {
+                    const int h = i / vec_per_row;
+                    const int e = (i - h * vec_per_row) * VEC;
+                    kv[u] = *reinterpret_cast<const Vec *>(ks + (int64_t)h * D + e);
+                    vv[u] = *reinterpret_cast<const Vec *>(vs + (int64_t)h * D + e);
+                }
+            }
+        };
+        load(lane);
         if (slot < 0)
             continue; // padding token: nothing is written
         if (slot >= n_slots) { // a slot outside the pool: nothing is written, the caller is told
@@ -46,16 +64,20 @@ __global__ void __launch_bounds__(256) kv_write_kernel(const uint16_t *__restric
         }
         const int64_t blk = slot / kBlockSize;
         const int off = (int)(slot % kBlockSize);
-        const uint16_t *ks = k_new + t * row_stride;
-        const uint16_t *vs = v_new + t * row_stride;
-        for (int i = lane; i < vec_per_tok; i += 32) {
-            const int h = i / vec_per_row;
-            const int e = (i - h * vec_per_row) * VEC;
-            const int64_t dst = blk * ((int64_t)Hkv * kBlockSize * D) + h * head_stride + off * tok_stride + e;
-            const Vec kv = *reinterpret_cast<const Vec *>(ks + (int64_t)h * D + e);
-            const Vec vv = *reinterpret_cast<const Vec *>(vs + (int64_t)h * D + e);
-            *reinterpret_cast<Vec *>(k_cache + dst) = kv;
-            *reinterpret_cast<Vec *>(v_cache + dst) = vv;
+        for (int i0 = lane; i0 < vec_per_tok; i0 += 4 * 32) {
+            if (i0 != lane)
+                load(i0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * 32;
+                if (i < vec_per_tok) {
+                    const int h = i / vec_per_row;
+                    const int e = (i - h * vec_per_row) * VEC;
+                    const int64_t dst = blk * ((int64_t)Hkv * kBlockSize * D) + h * head_stride + off * tok_stride + e;
+                    *reinterpret_cast<Vec *>(k_cache + dst) = kv[u];
+                    *reinterpret_cast<Vec *>(v_cache + dst) = vv[u];
+                }
+            }
         }
     }
 }

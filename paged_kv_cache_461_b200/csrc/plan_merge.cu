@@ -201,9 +201,11 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
     }
     // Split size of this step.  A decode CTA has a fixed cost (barrier setup, the first loads in
     // flight, the partial-state write and merge), so fewer, longer splits read HBM faster as long as
-    // there are still about a dozen CTAs per SM to balance.  The caller's explicit split is kept.
+    // there are still about a dozen CTAs per SM to balance.  A step with prefill work keeps the short
+    // split: its decode CTAs start on the SMs the prefill leaves free and spread over the others as
+    // the prefill CTAs finish, which short units fill more evenly.  The caller's explicit split is kept.
     int split = p.split_tokens;
-    if (p.auto_split) {
+    if (p.auto_split && carry_pf == 0) {
         const int64_t want = (int64_t)kDecCtasPerSm * p.num_sms;
         if ((int64_t)carry_u4 * p.Hkv >= want)
             split = s4;

@@ -97,11 +97,23 @@ enum PfBar {
     B_PF = 12,   // 2: P_X written (per tile, one arrival per row)
     B_OF = 14,   // 2: O_X of an item final (per tile)
     B_OE = 16,   // 2: O_X of an item read by the epilogue (per tile, one arrival per row)
-    B_LF = 18,   // 2: row sums and maxima of an item's tile X in shared memory (one arrival per row)
-    B_VFIX = 20, // V tail of an item zeroed
+    B_LF = 18,   // 2: row sums and maxima of an even item of tile X in shared memory (one arrival per row)
+    B_VFIX = 20, // V tail of an even tail-fixed item zeroed
     B_FIN = 21,
-    B_NUM = 22
+    B_LF1 = 22,  // 2: as B_LF, odd items of tile X
+    B_VFIX1 = 24, // as B_VFIX, odd tail-fixed items
+    B_NUM = 25
 };
+
+// The two signals without a reply of their own (the row sums for the epilogue, the zeroed V tail
+// for the MMA issuer) alternate between two barriers by item parity.  With one barrier a one-step
+// item could complete the next phase before the waiter had seen the previous one, and the waiter,
+// which tracks phases by parity, would then wait for good.  With two, the same barrier is reused two
+// items later, and by then the waiter has provably passed: the epilogue releases O_X (which the MMA
+// issuer waits for before the in-between item's first PV), and the V ring stage two steps back is
+// released only after the issuer's wait.
+__device__ __forceinline__ int bar_lf(int x, uint32_t item) { return ((item & 1) ? B_LF1 : B_LF) + x; }
+__device__ __forceinline__ int bar_vfix(uint32_t n) { return (n & 1) ? B_VFIX1 : B_VFIX; }
 
 constexpr uint32_t kTmemCols = 512;
 constexpr int kThreads = 512;
@@ -219,8 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             mbar_init(bar + (B_OF + s) * 8, 1);
             mbar_init(bar + (B_OE + s) * 8, kRowThreads);
             mbar_init(bar + (B_LF + s) * 8, kRowThreads);
+            mbar_init(bar + (B_LF1 + s) * 8, kRowThreads);
         }
         mbar_init(bar + B_VFIX * 8, 1);
+        mbar_init(bar + B_VFIX1 * 8, 1);
         mbar_init(bar + B_FIN * 8, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -249,8 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 tma_prefetch_desc(&tm_v);
             }
             bool ok = true;
-            uint32_t gs = 0; // K/V steps loaded so far by this CTA
-            uint32_t nq = 0; // items whose Q was loaded
+            uint32_t gs = 0;   // K/V steps loaded so far by this CTA
+            uint32_t nq = 0;   // items whose Q was loaded
+            uint32_t nfix = 0; // items whose V tail was zeroed
             for (int k = 0, item = snake_item(0, n_ctas); ok && item < n_items; item = snake_item(++k, n_ctas)) {
                 const ItemGeo g = item_geo(p, item);
                 // Q of this item, once the previous item's last QK^T has read the old Q
@@ -338,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0)
-                            mbar_arrive(bar + B_VFIX * 8);
+                            mbar_arrive(bar + bar_vfix(nfix) * 8);
+                        ++nfix;
                     }
                 }
             }
@@ -423,8 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     // a softmax's arrive to its PV issue is then a single barrier wait.
                     {
                         const bool fix = g.tail_fix && j == g.n_steps - 1;
-                        if (!mbar_wait_warp(bar + (fix ? B_VFIX : (B_VF + (gj & 1))) * 8,
-                                            fix ? (nfix & 1) : ((gj >> 1) & 1), abort_flag)) {
+                        if (!mbar_wait_warp(bar + (fix ? bar_vfix(nfix) : (B_VF + (gj & 1))) * 8,
+                                            fix ? ((nfix >> 1) & 1) : ((gj >> 1) & 1), abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -500,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 const TileGeo g = x ? gi.t1 : gi.t0;
                 if (g.rows == 0)
                     continue;
-                if (!mbar_wait_warp(bar + (B_LF + x) * 8, titem[x] & 1, abort_flag) ||
+                if (!mbar_wait_warp(bar + bar_lf(x, titem[x]) * 8, (titem[x] >> 1) & 1, abort_flag) ||
                     !mbar_wait_warp(bar + (B_OF + x) * 8, titem[x] & 1, abort_flag)) {
                     ok = false;
                     break;
@@ -659,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             float *slot = lm + (titem & 1) * 256;
             slot[row] = (la + lb) + (lc + ld);
             slot[128 + row] = m_ref;
-            mbar_arrive(bar + (B_LF + x) * 8);
+            mbar_arrive(bar + bar_lf(x, titem) * 8);
             ++titem;
         }
         if (!ok && lane == 0)

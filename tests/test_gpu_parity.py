@@ -341,8 +341,30 @@ def test_block_permutation_gives_bit_identical_output():
     st2 = DevStep(lay2, vals2)
     st2.write()
     out2, lse2 = st2.attend()
+    assert api.read_device_status(st.workspace) == 0 and api.read_device_status(st2.workspace) == 0
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
     assert torch.equal(lse1, lse2)
+
+
+def test_repeated_steps_are_bit_identical_and_clean():
+    # One-step prefill items (short chunks without context) mixed with long ones: the persistent
+    # prefill CTAs then finish some items' tiles while the previous item's other tile still runs, and
+    # every handoff between the warp roles must hold at any such timing.  Twenty calls on the same
+    # inputs: no status bit, and the same bits every time.
+    rng = np.random.default_rng(41)
+    chunks = [(int(n), 0) for n in rng.integers(20, 120, size=24)] + [(700, 900), (500, 0), (257, 1800)]
+    lay = _mixed_layout(41, n_dec=16, chunks=tuple(chunks))
+    vals = W.make_values_numpy(lay)
+    st = DevStep(lay, vals)
+    st.write()
+    ref, ref_lse = st.attend()
+    assert api.read_device_status(st.workspace) == 0
+    for _ in range(20):
+        out, lse = st.attend()
+        assert api.read_device_status(st.workspace) == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)) and torch.equal(lse, ref_lse)
+    o_ref, o_lse, _ = oracle_for_step(lay, vals)
+    assert_parity(ref, o_ref, ref_lse, o_lse, what="short and long prefill chunks")
 
 
 def test_shared_prefix_blocks_equal_private_copies_bit_exactly():
@@ -424,10 +446,13 @@ def test_split_and_unsplit_decode_agree():
 
 
 def _expected_split(lay, sms):
-    """The plan's per-step split rule restated on the host: 4x or 2x the 1024-key default while the
-    step's decode requests still give at least 12 split CTAs per SM, else the default."""
+    """The plan's per-step split rule restated on the host: in a step without prefill work, 4x or 2x
+    the 1024-key default while the step's decode requests still give at least 12 split CTAs per SM,
+    else the default."""
     L = (lay.ctx_lens + lay.q_lens).astype(np.int64)
     dec = (lay.q_lens > 0) & (lay.q_lens * (lay.num_q_heads // lay.num_kv_heads) <= 8)
+    if np.any((lay.q_lens > 0) & ~dec):
+        return 1024
     want = 12 * sms
     for split in (4096, 2048):
         if int(np.sum((L[dec] + split - 1) // split)) * lay.num_kv_heads >= want:
@@ -435,13 +460,17 @@ def _expected_split(lay, sms):
     return 1024
 
 
-@pytest.mark.parametrize("n_req,lo,hi", [(240, 100, 1000), (120, 2100, 3000), (12, 500, 9000)])
-def test_plan_picks_the_split_size_per_step(n_req, lo, hi):
-    # with the split left to the library the plan takes longer splits when the step has decode work
-    # enough to keep every SM busy with them; the result is bit-identical to asking for that split
+@pytest.mark.parametrize("n_req,lo,hi,n_pf", [(240, 100, 1000, 0), (120, 2100, 3000, 0), (12, 500, 9000, 0),
+                                               (240, 100, 1000, 1)])
+def test_plan_picks_the_split_size_per_step(n_req, lo, hi, n_pf):
+    # with the split left to the library the plan takes longer splits when a decode-only step has
+    # decode work enough to keep every SM busy with them (a step with a prefill chunk keeps the
+    # default); the result is bit-identical to asking for that split
     rng = np.random.default_rng(n_req)
     ctx = rng.integers(lo, hi, size=n_req)
-    lay = _layout("autosplit", ctx, np.ones(n_req, np.int32), 32, 8, 64, seed=n_req)
+    q = np.ones(n_req, np.int32)
+    q[:n_pf] = 300
+    lay = _layout("autosplit", ctx, q, 32, 8, 64, seed=n_req)
     vals = W.make_values_numpy(lay)
     st = DevStep(lay, vals)
     st.write()
