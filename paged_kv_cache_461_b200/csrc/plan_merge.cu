@@ -75,11 +75,13 @@ __device__ __forceinline__ void cta_excl_scan3(int a, int b, int c, int &ea, int
 // busy and the decode CTAs take every other SM, and all of them once prefill is done.  Rates
 // measured on B200 with this library's kernels running side by side (power-capped clocks):
 //   prefill  ~6.2 TFLOP/s per SM (925 TFLOP/s over 148 SMs alone);
-//   decode   ~65 GB/s per SM (two CTAs, ~190 KB of loads in flight per SM, so latency
+//   decode   ~80 GB/s per SM (three CTAs, ~190 KB of loads in flight per SM, so latency
 //            bound when confined to part of the GPU), at most the HBM rate.
+// (A forced sweep of the mixed 8192-token step put its optimum at 88-92 prefill SMs, where these
+// two rates balance.)
 constexpr float kPfFlopsPerSm = 6.2e12f;
 constexpr int kDecCtasPerSm = 12; // decode CTAs per SM below which the plan keeps the shorter split
-constexpr float kDecBytesPerSm = 65e9f;
+constexpr float kDecBytesPerSm = 80e9f;
 constexpr float kDecBytesMax = 6.35e12f;
 
 // Modelled step time (seconds) with pp prefill SMs out of num_sms: prefill lasts F / (pp f);
