@@ -121,9 +121,9 @@ constexpr int kRowThreads = 128; // one thread per query row of a tile
 // Registers per thread of each warpgroup after the split (the launch gives every thread
 // 65536 / 512 = 128): two softmax warpgroups hold a whole 128-key row of scores, the
 // epilogue and control warpgroups need little.
-constexpr int kRegSoftmax = 176;
-constexpr int kRegEpilogue = 80;
-constexpr int kRegControl = 72;
+constexpr int kRegSoftmax = 184;
+constexpr int kRegEpilogue = 72;
+constexpr int kRegControl = 64;
 constexpr int kRegSplit = kRowThreads * (2 * kRegSoftmax + kRegEpilogue + kRegControl);
 static_assert(kRegSplit <= 65536, "the warpgroup budgets must fit the CTA's register pool");
 
@@ -186,6 +186,38 @@ __device__ __forceinline__ int blocks_in_step(int n_keys, int j)
     return (min(kStepKeys, n_keys - j * kStepKeys) + kBlockSize - 1) / kBlockSize;
 }
 
+// P = exp2(s*c - m*c) of one thread's 128-score row -> bf16 pairs -> TMEM columns [0, 64) of its S (all of
+// S was read before), the row's sum added into two packed chains s2a / s2b; with MAX the row max of the scores is
+// taken alongside into m2 (two chains: few registers, and off the critical path behind the exponentials).
+template <bool MAX>
+__device__ __forceinline__ void softmax_exps(const uint32_t (&sv)[128], float c, float m_use, uint32_t tS,
+                                             uint64_t &s2a, uint64_t &s2b, float (&m2)[2])
+{
+    const uint64_t c2 = f2_pack(c, c);
+    const float nm = -m_use * c;
+    const uint64_t nm2 = f2_pack(nm, nm);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float s0 = __uint_as_float(sv[cc * 32 + 2 * i]);
+            const float s1 = __uint_as_float(sv[cc * 32 + 2 * i + 1]);
+            float e0, e1;
+            f2_unpack(f2_fma(f2_pack(s0, s1), c2, nm2), e0, e1);
+            const float p0 = fast_exp2(e0), p1 = fast_exp2(e1);
+            if (i & 1)
+                s2b = f2_add(s2b, f2_pack(p0, p1));
+            else
+                s2a = f2_add(s2a, f2_pack(p0, p1));
+            w[i] = pack_bf16x2(p0, p1);
+            if constexpr (MAX)
+                m2[i & 1] = fmax3(m2[i & 1], s0, s1);
+        }
+        tmem_st16(tS + cc * 16, w);
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                               const __grid_constant__ CUtensorMap tm_k,
@@ -193,7 +225,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                                                               const AttnParams p)
 {
     using Cfg = PfCfg<D>;
-    constexpr int kKS = D / 16; // k-steps of Q K^T
     const int n_items = (int)p.hdr->n_pf_tiles * p.Hkv;
     // CTAs that take work: the plan's share of the SMs for prefill (the rest go to decode)
     const int n_ctas = min(min((int)gridDim.x, n_items), max(1, (int)p.hdr->pf_ctas));
@@ -378,11 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     constexpr uint32_t H = Cfg::kHalfBytes >> 4;
                     umma_f16_x8_ss<0, 2, 4, 6, H, H + 2, H + 4, H + 6>(d_tmem, bq, bk, idesc_s, 0u);
                 } else {
-#pragma unroll
-                    for (int ks = 0; ks < kKS; ++ks) {
-                        const uint64_t off = (uint64_t)(((ks >> 2) * Cfg::kHalfBytes + (ks & 3) * 32) >> 4);
-                        umma_f16(d_tmem, bq + off, bk + off, idesc_s, ks > 0 ? 1u : 0u);
-                    }
+                    static_assert(D == 64, "head_dim 64 or 128");
+                    umma_f16_x4_ss<2, 4, 6>(d_tmem, bq, bk, idesc_s); // k-steps 0..3: +32 B in the swizzle row
                 }
                 umma_commit(bar + (B_SF + x) * 8);
             };
@@ -581,8 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 continue;
             const int p_row = row < g.rows ? g.p_min + row / G : g.p_max;
             float m_ref = -CUDART_INF_F;      // reference max, raw score units
-            uint64_t l2a = f2_pack(0.f, 0.f); // exact fp32 row sum, two packed chains
-            uint64_t l2b = f2_pack(0.f, 0.f);
+            uint64_t l2 = f2_pack(0.f, 0.f);  // exact fp32 row sum, two packed partial sums
             for (int j = 0; j < g.nkt; ++j, ++tstep) {
                 if (!mbar_wait_warp(bar + (B_SF + x) * 8, tstep & 1, abort_flag)) {
                     ok = false;
@@ -603,50 +630,38 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                         if (key0 + i > p_row)
                             sv[i] = __float_as_uint(-CUDART_INF_F);
                 }
-                // row max: eight independent chains, then combined
-                float m8[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
-#pragma unroll
-                for (int i = 16; i < 128; i += 16)
+                float alpha = 1.f;
+                uint64_t s2a = f2_pack(0.f, 0.f), s2b = s2a; // this step's row sum (two packed chains)
+                float m2[2] = {-CUDART_INF_F, -CUDART_INF_F};
+                if (j > 0) {
+                    // the exponentials against the reference max so far, with this step's row max taken
+                    // alongside; only if that grew past the threshold (rare) is the step redone max-first
+                    softmax_exps<true>(sv, c, m_ref, tS, s2a, s2b, m2);
+                    const float mx = fmaxf(m2[0], m2[1]);
+                    if (__any_sync(0xffffffffu, mx > m_ref + thresh)) {
+                        if (mx > m_ref + thresh) {
+                            alpha = fast_exp2((m_ref - mx) * c);
+                            m_ref = mx;
+                        }
+                        s2a = s2b = f2_pack(0.f, 0.f);
+                        tmem_wait_st(); // the first pass's P stores land before these replace them
+                        softmax_exps<false>(sv, c, m_ref, tS, s2a, s2b, m2);
+                    }
+                } else {
+                    // first step of the item: the row max first (eight independent chains, then combined)
+                    float m8[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        m8[q] = fmax3(m8[q], __uint_as_float(sv[i + 2 * q]), __uint_as_float(sv[i + 2 * q + 1]));
-                const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-                float alpha = 1.f;
-                if (j == 0) {
-                    m_ref = mx;
-                } else if (mx > m_ref + thresh) {
-                    alpha = fast_exp2((m_ref - mx) * c);
-                    m_ref = mx;
-                }
-                const uint64_t a2 = f2_pack(alpha, alpha);
-                l2a = f2_mul(l2a, a2);
-                l2b = f2_mul(l2b, a2);
-                // P = exp2(s*c - m*c) -> bf16 pairs -> TMEM columns [0, 64) of S_X (all of S was read above)
-                const uint64_t c2 = f2_pack(c, c);
-                const float nm = -m_ref * c;
-                const uint64_t nm2 = f2_pack(nm, nm);
+                        m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t w[16];
+                    for (int i = 16; i < 128; i += 16)
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float e0, e1;
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[cc * 32 + 2 * i]),
-                                                 __uint_as_float(sv[cc * 32 + 2 * i + 1])),
-                                         c2, nm2),
-                                  e0, e1);
-                        const float p0 = fast_exp2(e0), p1 = fast_exp2(e1);
-                        if (i & 1)
-                            l2b = f2_add(l2b, f2_pack(p0, p1));
-                        else
-                            l2a = f2_add(l2a, f2_pack(p0, p1));
-                        w[i] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(tS + cc * 16, w);
+                        for (int q = 0; q < 8; ++q)
+                            m8[q] = fmax3(m8[q], __uint_as_float(sv[i + 2 * q]), __uint_as_float(sv[i + 2 * q + 1]));
+                    m_ref = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+                    softmax_exps<false>(sv, c, m_ref, tS, s2a, s2b, m2);
                 }
+                l2 = f2_add(f2_mul(l2, f2_pack(alpha, alpha)), f2_add(s2a, s2b));
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
                     // O_X is stable (S_X(j) completing implies PV_X(j-1) completed) and PV_X(j)
                     // cannot start before the arrive below: rescale this thread's row
@@ -669,11 +684,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 break;
             // row sum and reference max -> the epilogue warpgroup (slot by item parity; the
             // epilogue reads it before it frees O_X, which this tile's next-but-one item waits for)
-            float la, lb, lc, ld;
-            f2_unpack(l2a, la, lb);
-            f2_unpack(l2b, lc, ld);
+            float la, lb;
+            f2_unpack(l2, la, lb);
             float *slot = lm + (titem & 1) * 256;
-            slot[row] = (la + lb) + (lc + ld);
+            slot[row] = la + lb;
             slot[128 + row] = m_ref;
             mbar_arrive(bar + bar_lf(x, titem) * 8);
             ++titem;

@@ -100,6 +100,25 @@ __device__ __forceinline__ void umma_f16_x8_ss(uint32_t d_tmem, uint64_t a, uint
     (void)A0;
 }
 
+// Four back-to-back kind::f16 MMAs into one accumulator, operands from shared memory, MMA i at
+// descriptors a + A_OFF(i) and b + A_OFF(i) (16-byte units, A_OFF(0) = 0); the first overwrites D.
+template <uint32_t A1, uint32_t A2, uint32_t A3>
+__device__ __forceinline__ void umma_f16_x4_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc)
+{
+    asm volatile(
+        "{\n\t.reg .pred pe;\n\t.reg .b64 ra, rb;\n\t.reg .b32 re;\n\t"
+        "elect.sync re|pe, 0xffffffff;\n\t"
+        "@pe tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 0;\n\t"
+        "add.s64 ra, %1, %4;\n\tadd.s64 rb, %2, %4;\n\t"
+        "@pe tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t"
+        "add.s64 ra, %1, %5;\n\tadd.s64 rb, %2, %5;\n\t"
+        "@pe tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t"
+        "add.s64 ra, %1, %6;\n\tadd.s64 rb, %2, %6;\n\t"
+        "@pe tcgen05.mma.cta_group::1.kind::f16 [%0], ra, rb, %3, 1;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "n"((uint64_t)A1), "n"((uint64_t)A2), "n"((uint64_t)A3)
+        : "memory");
+}
+
 // Eight back-to-back kind::f16 MMAs, A from TMEM (columns a_tmem + 8i), B from shared memory
 // (descriptor b + i * B_STEP in 16-byte units).
 template <uint32_t B_STEP>
