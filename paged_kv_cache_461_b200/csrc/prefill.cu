@@ -123,7 +123,7 @@ constexpr int kRowThreads = 128; // one thread per query row of a tile
 // epilogue and control warpgroups need little.
 constexpr int kRegSoftmax = 184;
 constexpr int kRegEpilogue = 72;
-constexpr int kRegControl = 64;
+constexpr int kRegControl = 72;
 constexpr int kRegSplit = kRowThreads * (2 * kRegSoftmax + kRegEpilogue + kRegControl);
 static_assert(kRegSplit <= 65536, "the warpgroup budgets must fit the CTA's register pool");
 
@@ -169,6 +169,26 @@ __device__ __forceinline__ ItemGeo item_geo(const AttnParams &p, int item)
     g.n_keys_all = (n1 ? g.t1.p_max : g.t0.p_max) + 1;
     g.tail_fix = (g.L % kBlockSize) != 0 && (g.n_keys_all - 1) / kBlockSize == (g.L - 1) / kBlockSize;
     return g;
+}
+
+// What the MMA issuer needs of an item (read one item ahead: item_geo's loads are two dependent
+// round trips to L2, which at an item boundary would stall the issuer while both tiles wait for S).
+struct MmaGeo {
+    int nkt[2], pmax[2], n_steps;
+    bool tail_fix;
+};
+
+__device__ __forceinline__ MmaGeo mma_geo(const AttnParams &p, int item)
+{
+    const ItemGeo g = item_geo(p, item);
+    MmaGeo m;
+    m.nkt[0] = g.t0.nkt;
+    m.nkt[1] = g.t1.nkt;
+    m.pmax[0] = g.t0.p_max;
+    m.pmax[1] = g.t1.p_max;
+    m.n_steps = g.n_steps;
+    m.tail_fix = g.tail_fix;
+    return m;
 }
 
 // The k-th work item of this CTA.  The work list is sorted by cost, most expensive
@@ -433,10 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             uint32_t nfix = 0;          // items with a zeroed V tail
             uint32_t tstep[2] = {0, 0}; // steps of tile X so far (phase of B_SF / B_PF)
             uint32_t titem[2] = {0, 0}; // items with tile X so far (phase of B_OF / B_OE)
+            MmaGeo next = mma_geo(p, snake_item(0, n_ctas)); // the CTA has at least one item
             for (int k = 0, item = snake_item(0, n_ctas); ok && item < n_items; item = snake_item(++k, n_ctas)) {
-                const ItemGeo g = item_geo(p, item);
-                const int nkt[2] = {g.t0.nkt, g.t1.nkt};
-                const int pmax[2] = {g.t0.p_max, g.t1.p_max};
+                const MmaGeo g = next;
+                const int nkt[2] = {g.nkt[0], g.nkt[1]};
+                const int pmax[2] = {g.pmax[0], g.pmax[1]};
                 if (!mbar_wait_warp(bar + B_Q * 8, nq & 1, abort_flag)) {
                     ok = false;
                     break;
@@ -460,6 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                         s_issued();
                     }
                 umma_commit(bar + (B_KE + (gs & 1)) * 8); // K of step 0 consumed
+                // the next item's geometry, while this item's first softmax runs
+                if (snake_item(k + 1, n_ctas) < n_items)
+                    next = mma_geo(p, snake_item(k + 1, n_ctas));
                 for (int j = 0; ok && j < g.n_steps; ++j) {
                     const uint32_t gj = gs + j;
                     // V of this step (loaded a step earlier, together with the K that S(j) used) and,
