@@ -330,7 +330,10 @@ cudaError_t launch_plan(const AttnParams &p, cudaStream_t s)
     if (n_buckets > 12 * 1024)
         n_buckets = 12 * 1024;
     const int smem = n_buckets * (int)sizeof(int);
-    plan_kernel<<<1, 1024, smem, s>>>(p, n_buckets);
+    // one thread per request (at least four warps, at most 1024 threads, which then loop): fewer warps make
+    // the block-wide scans and reductions of this short, latency-bound kernel cheaper
+    const int threads = min(1024, max(128, (p.num_seqs + 31) / 32 * 32));
+    plan_kernel<<<1, threads, smem, s>>>(p, n_buckets);
     return cudaGetLastError();
 }
 
