@@ -130,6 +130,12 @@ __global__ void gather_kernel(const uint16_t *__restrict__ cache, int64_t num_bl
 // stride over units and each CTA's threads over the unit's vectors, eight in flight per
 // thread.  PACK: cache -> staging (an id outside the pool gives zeros); otherwise
 // staging -> cache (an id outside the pool is skipped).
+// Resident copy CTAs per SM: 4 x 256 threads x 8 vectors of 16 bytes = 128 KB of loads in flight per SM.
+// Measured on B200 over 9,000 to 37,555 blocks: 6.26-6.53 TB/s read + written at 4 CTAs per SM against
+// 5.80-6.05 at 3, 6 or 8 (more bytes in flight are not faster here; a plain contiguous copy of the same bytes
+// runs at 6.66 TB/s).
+constexpr int kCopyCtasPerSm = 4;
+
 template <bool PACK>
 __global__ void __launch_bounds__(256) kv_block_copy_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                                                             int64_t num_blocks, int bv,
@@ -177,7 +183,7 @@ cudaError_t launch_kv_pack(const void *k_cache, const void *v_cache, int64_t num
                            const int32_t *ids, int num_ids, void *staging, int num_sms, cudaStream_t s)
 {
     const int64_t units = 2 * (int64_t)num_ids;
-    const unsigned grid = (unsigned)(units < (int64_t)num_sms * 8 ? units : (int64_t)num_sms * 8);
+    const unsigned grid = (unsigned)(units < (int64_t)num_sms * kCopyCtasPerSm ? units : (int64_t)num_sms * kCopyCtasPerSm);
     kv_block_copy_kernel<true><<<grid, 256, 0, s>>>(
         const_cast<uint4 *>(static_cast<const uint4 *>(k_cache)), const_cast<uint4 *>(static_cast<const uint4 *>(v_cache)),
         num_blocks, (int)(block_elems / 8), ids, units, static_cast<uint4 *>(staging));
@@ -188,7 +194,7 @@ cudaError_t launch_kv_unpack(const void *staging, const int32_t *ids, int num_id
                              int64_t num_blocks, int64_t block_elems, int num_sms, cudaStream_t s)
 {
     const int64_t units = 2 * (int64_t)num_ids;
-    const unsigned grid = (unsigned)(units < (int64_t)num_sms * 8 ? units : (int64_t)num_sms * 8);
+    const unsigned grid = (unsigned)(units < (int64_t)num_sms * kCopyCtasPerSm ? units : (int64_t)num_sms * kCopyCtasPerSm);
     kv_block_copy_kernel<false><<<grid, 256, 0, s>>>(static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache),
                                                      num_blocks, (int)(block_elems / 8), ids, units,
                                                      const_cast<uint4 *>(static_cast<const uint4 *>(staging)));
