@@ -5,13 +5,15 @@
 // K/V byte from HBM exactly once per kv head, with enough bytes in flight.
 //
 // Work unit = one CTA = (request r, kv head h, split s): keys
-// [s*S, min((s+1)*S, L_r)) of kv head h.  All G query heads of the group (and
+// [s*S, min((s+1)*S, L_r)) of kv head h, S the step's split size (the
+// caller's, or 1024 / 2048 / 4096 as the plan kernel chose it; read from the
+// workspace header).  All G query heads of the group (and
 // all query tokens of a short multi-token request) are packed as the N columns
 // of one warp MMA, so each K/V byte is read once per kv head.
 //
 // Data path per CTA (4 warps):
 //   * each warp owns every 4th 16-token block of the split and a private ring
-//     of 3 stages (2 when 16 rows are packed, so 3 CTAs fit per SM); lane 0
+//     of 2 stages (so 3 CTAs, 12 warps, fit per SM); lane 0
 //     fetches one (block, kv head) K tile and V tile with TMA loads (128-byte
 //     swizzled, 2 KiB per 64-column half) that complete on the stage's
 //     mbarrier, one ring ahead of use;
