@@ -19,14 +19,16 @@
 // warpgroups with setmaxnreg so that a softmax thread can hold a whole row):
 //   WG 0, WG 1  softmax of tile A and of tile B: one thread per query row
 //               (= TMEM lane), all 128 scores of a key step in registers after
-//               one tcgen05.ld pass.  Causal mask by select, row max over the
-//               thread's own registers, P = exp2(s*c - m*c) with packed fp32x2
-//               FMAs, bf16 P back into TMEM over S with tcgen05.st.  O is
-//               rescaled in TMEM only when a row's max grows by more than 2^8
-//               (a stale max leaves the normalised result unchanged).  After a
-//               tile's last step the row sum and max go to the epilogue
-//               warpgroup through shared memory and the softmax moves straight
-//               on to its next item.
+//               one tcgen05.ld pass.  Causal mask by select, P = exp2(s*c - m*c)
+//               with packed fp32x2 FMAs, bf16 P back into TMEM over S with
+//               tcgen05.st.  The reference max m moves (and O is rescaled in
+//               TMEM) only when a row's max grows by more than 2^8 (a stale max
+//               leaves the normalised result unchanged), so after an item's first
+//               step the exponentials run against the current m with the step's
+//               row max taken alongside, and a step is redone max-first only when
+//               that max passed the threshold.  After a tile's last step the row
+//               sum and max go to the epilogue warpgroup through shared memory
+//               and the softmax moves straight on to its next item.
 //   WG 2        epilogue of both tiles: waits for a tile's final O, writes O / l
 //               as bf16 (and the LSE), then frees O for the next item's first PV.
 //   WG 3        warp 12: TMA producer -- per item both Q tiles (3-D boxes
@@ -35,8 +37,8 @@
 //               tile and the V tile (8 paged blocks x 64-column halves, 2-D
 //               boxes) into separate 2-stage rings;
 //               warp 13: TMEM allocation (512 columns: S_A, O_A, S_B, O_B) and
-//               the MMAs (one elected lane issues, the warp stays converged), in
-//               the order
+//               the MMAs (one elected lane issues, the warp stays converged; it
+//               reads each item's geometry one item ahead), in the order
 //                 PV_A(j-1), S_A(j), PV_B(j-1), S_B(j)   (ping-pong)
 //               so the tensor core works on one tile while the other tile's
 //               softmax runs.  S = Q K^T is SS (both operands in smem);
