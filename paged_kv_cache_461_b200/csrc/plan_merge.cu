@@ -294,11 +294,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
         hdr->n_pf_tiles = (uint32_t)min((int64_t)carry_pf, p.max_pf_tiles);
         hdr->n_reduce = (uint32_t)carry_red;
         hdr->split_tokens = (uint32_t)split;
-#ifdef PA_FORCE_PF_CTAS
-        hdr->pf_ctas = (uint32_t)min(PA_FORCE_PF_CTAS, p.num_sms);
-#else
         hdr->pf_ctas = (uint32_t)pf_ctas;
-#endif
     }
 }
 
