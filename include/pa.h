@@ -89,9 +89,10 @@ typedef struct pa_cache_desc {
 typedef struct pa_attn_options {
     int32_t kv_split_tokens;       /* keys per split-KV partition of a decode request;
                                       a positive multiple of 16, used as given; 0 = the library
-                                      chooses per step on the device: 1024, or 2048 / 4096 when
-                                      the step's decode requests still give at least 12 split
-                                      CTAs per SM at that size (the workspace is sized for 1024) */
+                                      chooses per step on the device: 1024, or, in a step without
+                                      prefill work, 2048 / 4096 when the step's decode requests
+                                      still give at least 12 split CTAs per SM at that size (the
+                                      workspace is sized for 1024) */
     int32_t decode_max_query_len;  /* requests with q_len <= this take the memory-bound decode
                                       kernel instead of the tensor-core prefill kernel, e.g. k+1
                                       for speculative verification of k drafted tokens
