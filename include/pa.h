@@ -131,7 +131,7 @@ typedef struct pa_attn_options {
 #define PA_DEVICE_WAIT_TIMEOUT 4u /* a kernel gave up waiting on a copy or a tensor-core result */
 #define PA_DEVICE_BAD_SLOT 8u     /* pa_kv_write_ex: a slot >= num_blocks*block_size was skipped */
 
-PA_API int32_t pa_abi_version(void); /* 3 */
+PA_API int32_t pa_abi_version(void); /* 4 */
 PA_API const char *pa_status_string(pa_status_t status);
 
 /*
@@ -378,6 +378,36 @@ PA_API pa_status_t pa_attention_decode_fused(const void *q, int32_t num_q_heads,
                                              float softmax_scale, void *out, float *lse, void *workspace,
                                              size_t workspace_bytes, const pa_attn_options_t *options,
                                              pa_stream_t stream);
+
+/*
+ * pa_attention_mixed_write -- a whole step's KV write and attention, any
+ * step shape.  (hn.213312.xyz section 一, forward-pass paragraph: each step
+ * writes the new tokens' K/V into their slots, then attends over the cache.)
+ *
+ * Same arguments, rules and results as pa_attention_mixed_ex, plus this
+ * step's new rows k_new/v_new (bf16, token t's row at element
+ * t*new_row_stride, [Hkv, head_dim] contiguous) and slot_mapping (int64
+ * [num_tokens], as for pa_kv_write).  The rows are written by the same
+ * launch that plans the step (its first kernel: one CTA plans while the
+ * others write; neither reads what the other writes), so the plan costs no
+ * time of its own.  Cache bytes afterwards equal those of pa_kv_write with
+ * that slot mapping; out / lse are bit-identical to pa_kv_write followed by
+ * pa_attention_mixed_ex.  A slot outside the pool writes nothing and sets
+ * PA_DEVICE_BAD_SLOT in the status word at byte 0 of the workspace, beside
+ * the attention's own bits.  The workspace is sized by pa_workspace_size_ex.
+ * PA_ERR_INVALID_ARG for a NULL slot_mapping / k_new / v_new or
+ * new_row_stride < Hkv*head_dim.  (No counterpart on the pages: an engine
+ * entry point that folds the plan into the step's first kernel.)
+ */
+PA_API pa_status_t pa_attention_mixed_write(const void *q, int32_t num_q_heads, const void *k_new,
+                                            const void *v_new, int64_t new_row_stride, const int64_t *slot_mapping,
+                                            void *k_cache, void *v_cache, const pa_cache_desc_t *cache,
+                                            const int32_t *query_start_loc, const int32_t *seq_lens,
+                                            const int32_t *block_table, int32_t bt_stride, int32_t num_seqs,
+                                            int32_t num_tokens, int32_t max_query_len, int32_t max_seq_len,
+                                            float softmax_scale, void *out, float *lse, void *workspace,
+                                            size_t workspace_bytes, const pa_attn_options_t *options,
+                                            pa_stream_t stream);
 
 /*
  * pa_kv_pack / pa_kv_unpack -- copy whole cache blocks to and from a

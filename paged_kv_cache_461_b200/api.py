@@ -34,7 +34,7 @@ EXPORTED = ("pa_abi_version", "pa_status_string", "pa_kv_write", "pa_build_slot_
             "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack", "pa_merge_attn_states", "pa_debug_gather_kv",
             "pa_prefix_block_hashes", "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_cache_insert",
             "pa_prefix_cache_remove_block", "pa_prefix_cache_longest_hit", "pa_prefix_cache_size", "pa_kv_write_ex",
-            "pa_noalloc_device_status")
+            "pa_noalloc_device_status", "pa_attention_mixed_write")
 HASH_ALGOS = {"fnv1a64": 0, "sha256": 1}
 LAYOUT_HND = 0   # cache [num_blocks, num_kv_heads, 16, head_dim]
 LAYOUT_NHD = 1   # cache [num_blocks, 16, num_kv_heads, head_dim]
@@ -90,6 +90,9 @@ def lib():
         L.pa_attention_decode_fused.argtypes = [_vp, _i32, _vp, _vp, _i64, _vp, _vp, ctypes.POINTER(CacheDesc), _vp,
                                                 _vp, _vp, _i32, _i32, _i32, _i32, _i32, ctypes.c_float, _vp, _vp,
                                                 _vp, _sz, ctypes.POINTER(AttnOptions), _vp]
+        L.pa_attention_mixed_write.argtypes = [_vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp, ctypes.POINTER(CacheDesc),
+                                               _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, ctypes.c_float, _vp, _vp,
+                                               _vp, _sz, ctypes.POINTER(AttnOptions), _vp]
         L.pa_kv_pack.argtypes = [_vp, _vp, ctypes.POINTER(CacheDesc), _vp, _i32, _vp, _vp]
         L.pa_kv_unpack.argtypes = [_vp, _vp, _i32, _vp, _vp, ctypes.POINTER(CacheDesc), _vp]
         L.pa_merge_attn_states.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
@@ -109,7 +112,8 @@ def lib():
         L.pa_prefix_cache_size.argtypes = [_vp]
         L.pa_prefix_cache_size.restype = _i64
         for name in ("pa_kv_write", "pa_kv_write_ex", "pa_noalloc_device_status", "pa_build_slot_mapping", "pa_attention_mixed", "pa_attention_mixed_ex",
-                     "pa_attention_mixed_noalloc", "pa_attention_decode_fused", "pa_kv_pack", "pa_kv_unpack",
+                     "pa_attention_mixed_noalloc", "pa_attention_decode_fused", "pa_attention_mixed_write",
+                     "pa_kv_pack", "pa_kv_unpack",
                      "pa_merge_attn_states", "pa_debug_gather_kv"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -358,6 +362,45 @@ def attention_mixed(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
                                        float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(),
                                        ctypes.byref(o) if o else None, st), "pa_attention_mixed")
+    return out
+
+
+def attention_mixed_write(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                          k_cache: torch.Tensor, v_cache: torch.Tensor, query_start_loc: torch.Tensor,
+                          seq_lens: torch.Tensor, block_table: torch.Tensor, max_query_len: int, max_seq_len: int,
+                          softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                          lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                          kv_split_tokens: int = 0, decode_max_query_len: int = 0, stream=None,
+                          layout: str = "HND", concurrent: bool = True) -> torch.Tensor:
+    """pa_attention_mixed_write: kv_write(k_new, v_new, slot_mapping) and attention_mixed in one call, the
+    write and the step's plan in one launch (k_new/v_new [T, Hkv, D], rows may be strided; slot_mapping
+    int64 [T])."""
+    _need_q_out(q, out, lse)
+    _need_caches(k_cache, v_cache, q.device)
+    _need_meta(query_start_loc, seq_lens, block_table, q.device)
+    d = cache_desc(k_cache, layout)
+    row_stride = _need_new_rows(k_new, v_new, d, q.device)
+    T, Hq, D = q.shape
+    R = seq_lens.shape[0]
+    if k_new.shape[0] != T:
+        raise ValueError(f"k_new has {k_new.shape[0]} rows, q has {T} tokens")
+    _need(slot_mapping, torch.int64, "slot_mapping", shape=(T,), dense=True, device=q.device)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(R, T, Hq, k_cache, max_seq_len, kv_split_tokens, decode_max_query_len, layout)
+    _need(workspace, torch.uint8, "workspace", dense=True, device=q.device)
+    st = _stream(stream, q.device)
+    fork = concurrent and _may_fork(Hq, k_cache, layout, max_query_len, decode_max_query_len)
+    o = _opts(kv_split_tokens, decode_max_query_len, (st.value or 0) if fork else None)
+    _check(lib().pa_attention_mixed_write(_ptr(q), Hq, _ptr(k_new), _ptr(v_new), row_stride, _ptr(slot_mapping),
+                                          _ptr(k_cache), _ptr(v_cache), ctypes.byref(d), _ptr(query_start_loc),
+                                          _ptr(seq_lens), _ptr(block_table), block_table.stride(0), R, T,
+                                          int(max_query_len), int(max_seq_len), float(softmax_scale), _ptr(out),
+                                          _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          ctypes.byref(o) if o else None, st), "pa_attention_mixed_write")
     return out
 
 

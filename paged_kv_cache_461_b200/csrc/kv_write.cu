@@ -14,72 +14,20 @@
 // forward pass writes each layer's new K/V into the cache before attention.
 #include <type_traits>
 
+#include "kv_write.cuh"
 #include "pa_internal.cuh"
 
 namespace pa {
 namespace {
 
-// One warp per token; lanes stride over the token's Hkv*D/VEC vectors of K and V.
+// One warp per token (kv_write.cuh); a slot outside the pool sets PA_DEVICE_BAD_SLOT in *status.
 template <int VEC>
-__global__ void __launch_bounds__(256) kv_write_kernel(const uint16_t *__restrict__ k_new,
-                                                       const uint16_t *__restrict__ v_new, int64_t row_stride,
-                                                       const int64_t *__restrict__ slots, int num_tokens,
-                                                       uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
-                                                       int64_t num_blocks, int Hkv, int D, int head_stride,
-                                                       int tok_stride, uint32_t *status)
+__global__ void __launch_bounds__(256) kv_write_kernel(const KvWriteArgs a, uint32_t *status)
 {
-    using Vec = typename std::conditional<VEC == 8, uint4, uint16_t>::type;
-    const int lane = threadIdx.x & 31;
-    const int warps_per_cta = blockDim.x >> 5;
-    const int64_t n_slots = num_blocks * kBlockSize;
-    const int vec_per_row = D / VEC;
-    const int vec_per_tok = Hkv * vec_per_row;
-    for (int64_t t = (int64_t)blockIdx.x * warps_per_cta + (threadIdx.x >> 5); t < num_tokens;
-         t += (int64_t)gridDim.x * warps_per_cta) {
-        const int64_t slot = slots[t];
-        const uint16_t *ks = k_new + t * row_stride;
-        const uint16_t *vs = v_new + t * row_stride;
-        // Up to four vectors of K and four of V per lane: the first group is loaded before the
-        // slot is known (the token's rows are always readable), so the two loads overlap.
-        Vec kv[4], vv[4];
-        auto load = [&](int i0) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = i0 + u * 32;
-                if (i < vec_per_tok) {
-                    const int h = i / vec_per_row;
-                    const int e = (i - h * vec_per_row) * VEC;
-                    kv[u] = *reinterpret_cast<const Vec *>(ks + (int64_t)h * D + e);
-                    vv[u] = *reinterpret_cast<const Vec *>(vs + (int64_t)h * D + e);
-                }
-            }
-        };
-        load(lane);
-        if (slot < 0)
-            continue; // padding token: nothing is written
-        if (slot >= n_slots) { // a slot outside the pool: nothing is written, the caller is told
-            if (status != nullptr && lane == 0)
-                atomicOr(status, PA_DEVICE_BAD_SLOT);
-            continue;
-        }
-        const int64_t blk = slot / kBlockSize;
-        const int off = (int)(slot % kBlockSize);
-        for (int i0 = lane; i0 < vec_per_tok; i0 += 4 * 32) {
-            if (i0 != lane)
-                load(i0);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = i0 + u * 32;
-                if (i < vec_per_tok) {
-                    const int h = i / vec_per_row;
-                    const int e = (i - h * vec_per_row) * VEC;
-                    const int64_t dst = blk * ((int64_t)Hkv * kBlockSize * D) + h * head_stride + off * tok_stride + e;
-                    *reinterpret_cast<Vec *>(k_cache + dst) = kv[u];
-                    *reinterpret_cast<Vec *>(v_cache + dst) = vv[u];
-                }
-            }
-        }
-    }
+    kv_write_tokens<VEC>(a, blockIdx.x, gridDim.x, [&]() {
+        if (status != nullptr)
+            atomicOr(status, PA_DEVICE_BAD_SLOT);
+    });
 }
 
 // One CTA per request; threads stride over its query rows.
@@ -205,28 +153,14 @@ cudaError_t launch_kv_write(const void *k_new, const void *v_new, int64_t row_st
                             int num_tokens, void *k_cache, void *v_cache, int64_t num_blocks, int Hkv, int D,
                             int nhd, uint32_t *status, cudaStream_t s)
 {
-    const int head_stride = nhd ? D : kBlockSize * D;
-    const int tok_stride = nhd ? Hkv * D : D;
-    const bool vec_ok = ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new) |
-                          reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) % 16 == 0) &&
-                        (row_stride % 8 == 0) && (D % 8 == 0);
-    const int threads = 256;
-    const int warps = threads / 32;
-    int64_t blocks = ((int64_t)num_tokens + warps - 1) / warps;
-    if (blocks > 148 * 16)
-        blocks = 148 * 16;
-    if (blocks < 1)
-        blocks = 1;
+    bool vec_ok = false;
+    const KvWriteArgs a =
+        kv_write_args(k_new, v_new, row_stride, slots, num_tokens, k_cache, v_cache, num_blocks, Hkv, D, nhd, &vec_ok);
+    const unsigned blocks = (unsigned)kv_write_ctas(num_tokens);
     if (vec_ok)
-        kv_write_kernel<8><<<(unsigned)blocks, threads, 0, s>>>(
-            static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new), row_stride, slots, num_tokens,
-            static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache), num_blocks, Hkv, D, head_stride,
-            tok_stride, status);
+        kv_write_kernel<8><<<blocks, 256, 0, s>>>(a, status);
     else
-        kv_write_kernel<1><<<(unsigned)blocks, threads, 0, s>>>(
-            static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new), row_stride, slots, num_tokens,
-            static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache), num_blocks, Hkv, D, head_stride,
-            tok_stride, status);
+        kv_write_kernel<1><<<blocks, 256, 0, s>>>(a, status);
     return cudaGetLastError();
 }
 

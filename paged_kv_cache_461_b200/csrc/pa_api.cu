@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "kv_write.cuh"
 #include "pa_internal.cuh"
 
 using namespace pa;
@@ -218,7 +219,7 @@ struct NvtxRange {
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 3; }
+int32_t pa_abi_version(void) { return 4; }
 
 const char *pa_status_string(pa_status_t s)
 {
@@ -302,9 +303,13 @@ size_t pa_workspace_size(int32_t num_seqs, int32_t num_tokens, int32_t num_q_hea
 namespace {
 
 // New K/V rows the decode kernel stores itself (pa_attention_decode_fused).
+// The step's new K/V rows, written by the attention call itself: with slots == nullptr by the decode
+// kernel (decode-shaped steps, slots from the block tables), else by the launch that also plans the step
+// (any step, through the given slot mapping).
 struct FusedWrite {
     const void *k_new, *v_new;
     int64_t row_stride;
+    const int64_t *slots;
 };
 
 pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cache, const void *v_cache,
@@ -351,7 +356,7 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
 
     const int Hkv = cache->num_kv_heads;
     const bool nhd = cache->layout == PA_LAYOUT_NHD;
-    if (fw) {
+    if (fw && !fw->slots) {
         // every request must be decode-shaped: the prefill kernel reads the new rows from the cache
         if ((int64_t)max_query_len * P.G > P.dec_rows_cap || P.NT == 0)
             return PA_ERR_UNSUPPORTED;
@@ -360,6 +365,8 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
         if (!aligned16(fw->k_new) || !aligned16(fw->v_new) || fw->row_stride % 8 != 0)
             return PA_ERR_UNSUPPORTED;
     }
+    if (fw && fw->slots && (!fw->k_new || !fw->v_new || fw->row_stride < (int64_t)Hkv * D))
+        return PA_ERR_INVALID_ARG;
     // HND: 2-D {D, blocks*Hkv*16} with 16-row boxes;  NHD: 3-D {D, Hkv, blocks*16} with {64, 1, 16} boxes
     const uint64_t kv_rows = (uint64_t)cache->num_blocks * Hkv * kBlockSize;
     const uint64_t tok_rows = (uint64_t)cache->num_blocks * kBlockSize;
@@ -405,7 +412,7 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     p.QD = P.QD;
     p.dec_rows_cap = P.dec_rows_cap;
     p.nhd = nhd;
-    if (fw) {
+    if (fw && !fw->slots) {
         p.k_new = static_cast<const uint16_t *>(fw->k_new);
         p.v_new = static_cast<const uint16_t *>(fw->v_new);
         p.new_row_stride = fw->row_stride;
@@ -426,8 +433,18 @@ pa_status_t attention_impl(const void *q, int32_t num_q_heads, const void *k_cac
     // rows.  Without a side stream prefill takes every SM and decode follows it on `stream`.
     const bool fork = prefill && P.NT > 0 && side != nullptr;
     p.pf_all_sms = fork ? 0 : 1;
-    NvtxRange range(fw ? "pa_attention_decode_fused" : "pa_attention_mixed");
-    cudaError_t e = launch_plan(p, s);
+    NvtxRange range(!fw ? "pa_attention_mixed" : fw->slots ? "pa_attention_mixed_write" : "pa_attention_decode_fused");
+    cudaError_t e;
+    if (fw && fw->slots) {
+        // the step's KV write and its plan in one launch (neither reads what the other writes)
+        bool vec_ok = false;
+        const KvWriteArgs w = kv_write_args(fw->k_new, fw->v_new, fw->row_stride, fw->slots, num_tokens,
+                                            const_cast<void *>(k_cache), const_cast<void *>(v_cache),
+                                            cache->num_blocks, Hkv, D, nhd, &vec_ok);
+        e = launch_write_plan(p, w, vec_ok, s);
+    } else {
+        e = launch_plan(p, s);
+    }
     if (e != cudaSuccess)
         return PA_ERR_CUDA;
     if (fork && (cudaEventRecord(ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess))
@@ -474,7 +491,24 @@ pa_status_t pa_attention_decode_fused(const void *q, int32_t num_q_heads, const 
                                       void *workspace, size_t workspace_bytes, const pa_attn_options_t *options,
                                       pa_stream_t stream)
 {
-    const FusedWrite fw{k_new, v_new, new_row_stride};
+    const FusedWrite fw{k_new, v_new, new_row_stride, nullptr};
+    return attention_impl(q, num_q_heads, k_cache, v_cache, cache, query_start_loc, seq_lens, block_table, bt_stride,
+                          num_seqs, num_tokens, max_query_len, max_seq_len, softmax_scale, out, lse, workspace,
+                          workspace_bytes, options, &fw, stream);
+}
+
+pa_status_t pa_attention_mixed_write(const void *q, int32_t num_q_heads, const void *k_new, const void *v_new,
+                                     int64_t new_row_stride, const int64_t *slot_mapping, void *k_cache,
+                                     void *v_cache, const pa_cache_desc_t *cache, const int32_t *query_start_loc,
+                                     const int32_t *seq_lens, const int32_t *block_table, int32_t bt_stride,
+                                     int32_t num_seqs, int32_t num_tokens, int32_t max_query_len,
+                                     int32_t max_seq_len, float softmax_scale, void *out, float *lse,
+                                     void *workspace, size_t workspace_bytes, const pa_attn_options_t *options,
+                                     pa_stream_t stream)
+{
+    if (!slot_mapping)
+        return PA_ERR_INVALID_ARG;
+    const FusedWrite fw{k_new, v_new, new_row_stride, slot_mapping};
     return attention_impl(q, num_q_heads, k_cache, v_cache, cache, query_start_loc, seq_lens, block_table, bt_stride,
                           num_seqs, num_tokens, max_query_len, max_seq_len, softmax_scale, out, lse, workspace,
                           workspace_bytes, options, &fw, stream);

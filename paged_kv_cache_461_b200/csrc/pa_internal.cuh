@@ -25,7 +25,8 @@ struct WsHeader {
     uint32_t n_reduce;    // decode requests with more than one split (merged by their last split CTA)
     uint32_t pf_ctas;     // persistent prefill CTAs that take work; the others leave their SM to decode
     uint32_t split_tokens; // keys per split-KV partition of this step's decode requests
-    uint32_t pad[58];
+    uint32_t write_epoch;  // call id published once the status word is cleared (write-and-plan launch)
+    uint32_t pad[57];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -92,6 +93,8 @@ cudaError_t launch_slot_mapping(const int32_t *qsl, const int32_t *seq_lens, con
 cudaError_t launch_gather(const void *cache, int64_t num_blocks, int Hkv, int D, int nhd, const int32_t *bt_row,
                           int seq_len, void *out, cudaStream_t s);
 cudaError_t launch_plan(const AttnParams &p, cudaStream_t s);
+struct KvWriteArgs;
+cudaError_t launch_write_plan(const AttnParams &p, const KvWriteArgs &w, bool vec_ok, cudaStream_t s);
 cudaError_t launch_decode(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int NT,
                           int64_t grid_units, cudaStream_t s);
 cudaError_t launch_merge_states(const float *part_out, const float *part_lse, const int32_t *parts_per_row,

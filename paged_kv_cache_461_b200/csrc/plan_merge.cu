@@ -13,10 +13,13 @@
 // Inside a step the split-KV merge runs at the end of the decode kernel itself.
 #include <math_constants.h>
 
+#include <atomic>
 #include <type_traits>
 
+#include "kv_write.cuh"
 #include "merge.cuh"
 #include "pa_internal.cuh"
+#include "ptx.cuh"
 
 namespace pa {
 namespace {
@@ -135,12 +138,13 @@ __device__ __forceinline__ int pair_cost(int ctx, int q_len, int qp, int tq)
 // histogram, so the persistent prefill CTAs, which walk the list in snake order, end
 // at nearly the same time.  Pairs of equal cost land in any order; every pair is
 // computed independently, so the order never changes a result.
-__global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_buckets)
+// hist: [n_buckets] ints of dynamic shared memory (pair counts, then start offsets).  Called by every
+// thread of one CTA.  reset_status: clear the status word first (the caller did otherwise).
+__device__ __forceinline__ void plan_body(const AttnParams &p, int n_buckets, int *hist, bool reset_status)
 {
-    extern __shared__ int hist[]; // [n_buckets] pair counts, then start offsets
     __shared__ unsigned long long s_sum[2][32];
     WsHeader *hdr = p.hdr;
-    if (threadIdx.x == 0)
+    if (reset_status && threadIdx.x == 0)
         hdr->status = 0u;
     // work estimates, per thread then reduced once: keys read by its decode requests and
     // causal (query, key) pairs of its prefill requests
@@ -298,6 +302,40 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
     }
 }
 
+__global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_buckets)
+{
+    extern __shared__ int hist[];
+    plan_body(p, n_buckets, hist, true);
+}
+
+// One launch for the start of a step: CTA 0 plans the step's attention while the other CTAs write its new
+// K/V rows into the cache (neither reads what the other writes).  A slot outside the pool sets
+// PA_DEVICE_BAD_SLOT in the status word, which CTA 0 clears for this call first: a writer that meets one
+// waits (bounded) until CTA 0 has published this call's epoch after the clear.
+template <int VEC>
+__global__ void __launch_bounds__(256) write_plan_kernel(const AttnParams p, int n_buckets, const KvWriteArgs w,
+                                                         uint32_t epoch)
+{
+    extern __shared__ int hist[];
+    WsHeader *hdr = p.hdr;
+    if (blockIdx.x == 0) {
+        if (threadIdx.x == 0) {
+            hdr->status = 0u;
+            __threadfence();
+            atomicExch(&hdr->write_epoch, epoch);
+        }
+        plan_body(p, n_buckets, hist, false);
+        return;
+    }
+    kv_write_tokens<VEC>(w, blockIdx.x - 1, gridDim.x - 1, [&]() {
+        const uint64_t t0 = global_timer_ns();
+        for (int it = 0; it < (1 << 20); ++it)
+            if (atomicAdd(&hdr->write_epoch, 0u) == epoch || global_timer_ns() - t0 > kWaitLimitNs)
+                break;
+        atomicOr(&hdr->status, PA_DEVICE_BAD_SLOT);
+    });
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) merge_states_kernel(const float *__restrict__ part_out,
                                                            const float *__restrict__ part_lse,
@@ -330,6 +368,22 @@ cudaError_t launch_plan(const AttnParams &p, cudaStream_t s)
     // the block-wide scans and reductions of this short, latency-bound kernel cheaper
     const int threads = min(1024, max(128, (p.num_seqs + 31) / 32 * 32));
     plan_kernel<<<1, threads, smem, s>>>(p, n_buckets);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_write_plan(const AttnParams &p, const KvWriteArgs &w, bool vec_ok, cudaStream_t s)
+{
+    int n_buckets = p.max_seq_len / 128 + 2;
+    if (n_buckets > 12 * 1024)
+        n_buckets = 12 * 1024;
+    const int smem = n_buckets * (int)sizeof(int);
+    static std::atomic<uint32_t> epoch_counter{0};
+    const uint32_t epoch = ++epoch_counter;
+    const unsigned grid = 1u + (unsigned)kv_write_ctas(w.num_tokens);
+    if (vec_ok)
+        write_plan_kernel<8><<<grid, 256, smem, s>>>(p, n_buckets, w, epoch);
+    else
+        write_plan_kernel<1><<<grid, 256, smem, s>>>(p, n_buckets, w, epoch);
     return cudaGetLastError();
 }
 

@@ -32,7 +32,7 @@ int main(void)
     CHECK(sizeof(pa_cache_desc_t) == 24);
     CHECK(sizeof(pa_attn_options_t) == 32 + 3 * sizeof(void *));
     CHECK(sizeof(pa_block_hash_t) == 32);
-    CHECK(pa_abi_version() == 3);
+    CHECK(pa_abi_version() == 4);
     CHECK(strcmp(pa_status_string(PA_ERR_WORKSPACE_TOO_SMALL), "PA_ERR_WORKSPACE_TOO_SMALL") == 0);
 
     memset(&d, 0, sizeof d);

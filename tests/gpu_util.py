@@ -120,6 +120,21 @@ class DevStep:
         return out, lse
 
 
+def write_and_attend_mixed(st: "DevStep", kv_split_tokens=0, with_lse=True, scale=None, workspace=None,
+                           decode_max_query_len=0):
+    """pa_attention_mixed_write on a DevStep: its K/V written (through its slot mapping) by the launch that
+    also plans the step, then attention as attention_mixed does."""
+    lay = st.layout
+    out, lse = st._outs(with_lse)
+    workspace = st._ws(workspace, kv_split_tokens, decode_max_query_len)
+    api.attention_mixed_write(st.q, st.k_new, st.v_new, st.slots, st.k_cache, st.v_cache, st.qsl, st.seq_lens,
+                              st.bt, lay.max_query_len, lay.max_seq_len, softmax_scale=scale, out=out, lse=lse,
+                              workspace=workspace, kv_split_tokens=kv_split_tokens,
+                              decode_max_query_len=decode_max_query_len, layout=st.kv_layout)
+    st.workspace = workspace
+    return out, lse
+
+
 def work_counts(workspace: torch.Tensor):
     """(decode units, prefill work items, split requests) the plan kernel wrote into the workspace header."""
     h = workspace[:16].view(torch.int32).cpu().tolist()

@@ -47,7 +47,7 @@ def test_library_exports_nothing_else(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.pa_abi_version() == 3
+    assert L.pa_abi_version() == 4
     for code, name in api.STATUS_NAMES.items():
         assert L.pa_status_string(code).decode() == name
 
@@ -233,6 +233,28 @@ def test_fused_decode_host_validation(L):
     assert _fused(L, stride=1028) == 2                   # not a multiple of 8 elements
     assert _fused(L, kn=FAKE + (1 << 33) + 2) == 2       # k_new not 16-byte aligned
     assert _fused(L, hq=8 * 3) == 2
+
+
+def _mixed_write(L, **kw):
+    a = dict(q=FAKE, hq=32, kn=FAKE + (1 << 33), vn=FAKE + (1 << 33) + (1 << 28), stride=1024,
+             slots=FAKE + (1 << 34), k=FAKE + (1 << 31), v=FAKE + (1 << 31) + (1 << 29), desc=_desc(), qsl=FAKE,
+             sl=FAKE, bt=FAKE, bts=64, R=4, T=4, mq=300, ms=1000, scale=0.088, out=FAKE + (1 << 30), lse=None,
+             ws=FAKE + (1 << 32), wsb=1 << 30, opt=None)
+    a.update(kw)
+    return L.pa_attention_mixed_write(a["q"], a["hq"], a["kn"], a["vn"], a["stride"], a["slots"], a["k"], a["v"],
+                                      ctypes.byref(a["desc"]), a["qsl"], a["sl"], a["bt"], a["bts"], a["R"], a["T"],
+                                      a["mq"], a["ms"], ctypes.c_float(a["scale"]), a["out"], a["lse"], a["ws"],
+                                      a["wsb"], a["opt"], None)
+
+
+def test_mixed_write_host_validation(L):
+    # the write-and-plan entry point takes any step shape (here prefill-shaped requests), and checks
+    # its write arguments before anything is enqueued
+    assert _mixed_write(L, slots=None) == 1
+    assert _mixed_write(L, kn=None) == 1
+    assert _mixed_write(L, stride=1000) == 1             # < Hkv * D
+    assert _mixed_write(L, wsb=16) == 3                  # workspace too small
+    assert _mixed_write(L, R=0) == 0
 
 
 def test_binding_rejects_host_tensors_before_the_library(L):

@@ -15,7 +15,7 @@ import oracle
 from paged_kv_cache_461_b200 import api, build
 from paged_kv_cache_461_b200 import workloads as W
 from tests.gpu_util import (DevStep, assert_parity, oracle_for_step, to_dev_bf16, to_hnd, to_host_bits, to_nhd,
-                            work_counts)
+                            work_counts, write_and_attend_mixed)
 
 pytestmark = pytest.mark.gpu
 
@@ -157,6 +157,88 @@ def test_fused_decode_full_size_llama3_8b_decode():
     assert api.read_device_status(st.workspace) == 0
     assert _bits_equal(out_f, out_u) and torch.equal(lse_f, lse_u)
     assert _bits_equal(st.k_cache, k_written)
+
+
+# ----------------------------------------------------------------------------- KV write + plan in one launch
+
+MIXED_WRITE_CASES = [
+    # (D, Hq, Hkv, q lens of the chunks, n decodes, layout, padding tokens)
+    (128, 32, 8, (300, 129, 64, 1), 24, "HND", False),
+    (128, 32, 8, (257, 40), 8, "NHD", True),
+    (64, 16, 4, (200, 33), 12, "HND", True),
+    (128, 32, 8, (), 40, "HND", False),          # decode only
+    (128, 32, 8, (500, 300), 0, "HND", False),   # prefill only
+]
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,chunks,n_dec,kv_layout,pad", MIXED_WRITE_CASES)
+def test_mixed_write_equals_write_then_attend(D, Hq, Hkv, chunks, n_dec, kv_layout, pad):
+    # pa_attention_mixed_write writes the step's rows in the launch that plans the step: the cache bytes
+    # equal the oracle's KV write, the outputs pa_kv_write + pa_attention_mixed_ex bit for bit
+    rng = np.random.default_rng(D + Hq + n_dec + len(chunks))
+    ctx = list(rng.integers(0, 1500, size=n_dec)) + [int(c) for c in rng.integers(0, 900, size=len(chunks))]
+    q = [1] * n_dec + list(chunks)
+    lay = _layout("mixw", ctx, q, Hq, Hkv, D, seed=int(sum(ctx)) % 977)
+    vals = W.make_values_numpy(lay, sentinel="pattern")
+    slots = lay.slot_mapping.copy()
+    if pad:
+        slots[rng.random(len(slots)) < 0.1] = -1          # padding tokens: nothing written for them
+    ref_st = DevStep(lay, vals, kv_layout=kv_layout)
+    ref_st.slots = torch.from_numpy(slots).cuda()
+    ref_st.write()
+    out_u, lse_u = ref_st.attend()
+    st = DevStep(lay, vals, kv_layout=kv_layout)
+    st.slots = torch.from_numpy(slots).cuda()
+    out_w, lse_w = write_and_attend_mixed(st)
+    torch.cuda.synchronize()
+    assert api.read_device_status(st.workspace) == 0
+    assert _bits_equal(out_w, out_u), "output differs from write-then-attend"
+    assert torch.equal(lse_w, lse_u)
+    kc, vc = oracle.kv_write(vals.k_new, vals.v_new, slots, vals.k_cache, vals.v_cache)
+    k_dev = to_hnd(st.k_cache) if kv_layout == "NHD" else st.k_cache
+    v_dev = to_hnd(st.v_cache) if kv_layout == "NHD" else st.v_cache
+    assert np.array_equal(to_host_bits(k_dev), kc)
+    assert np.array_equal(to_host_bits(v_dev), vc)
+    if not pad:
+        ref, ref_lse, _ = oracle_for_step(lay, vals)
+        assert_parity(out_w, ref, lse_w, ref_lse, what=f"mixed write D{D} {kv_layout} chunks{chunks}")
+
+
+def test_mixed_write_reports_slots_outside_the_pool():
+    lay = _layout("mixwb", [100, 200, 0], [1, 1, 90], 32, 8, 128, seed=5)
+    vals = W.make_values_numpy(lay, sentinel="pattern")
+    st = DevStep(lay, vals)
+    slots = lay.slot_mapping.copy()
+    slots[1] = lay.num_blocks * 16 + 5                    # outside the pool: not written, reported
+    st.slots = torch.from_numpy(slots).cuda()
+    for _ in range(3):                                    # the bit belongs to each call, set again each time
+        write_and_attend_mixed(st)
+        torch.cuda.synchronize()
+        assert api.read_device_status(st.workspace) & api.DEVICE_BAD_SLOT
+    ok = lay.slot_mapping.copy()
+    st.slots = torch.from_numpy(ok).cuda()
+    write_and_attend_mixed(st)                            # a clean call clears it
+    torch.cuda.synchronize()
+    assert api.read_device_status(st.workspace) == 0
+    kc, _ = oracle.kv_write(vals.k_new, vals.v_new, ok, vals.k_cache, vals.v_cache)
+    assert np.array_equal(to_host_bits(st.k_cache), kc)
+
+
+def test_mixed_write_full_size_mixed_step_8192():
+    lay = W.workload_layout("mixed_step_8192")
+    vals = W.make_values_torch(lay, "cuda")
+    k0, v0 = vals.k_cache.clone(), vals.v_cache.clone()
+    st = DevStep(lay, vals)
+    st.write()
+    out_u, lse_u = st.attend()
+    k_written, v_written = st.k_cache.clone(), st.v_cache.clone()
+    st.k_cache.copy_(k0)
+    st.v_cache.copy_(v0)
+    out_w, lse_w = write_and_attend_mixed(st)
+    torch.cuda.synchronize()
+    assert api.read_device_status(st.workspace) == 0
+    assert _bits_equal(out_w, out_u) and torch.equal(lse_w, lse_u)
+    assert _bits_equal(st.k_cache, k_written) and _bits_equal(st.v_cache, v_written)
 
 
 # ----------------------------------------------------------------------------- block pack / unpack
