@@ -134,17 +134,19 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
                 atomicOr(&p.hdr->status, PA_DEVICE_BAD_BLOCK);
             mbar_arrive_expect_tx(bar, Cfg::kStage);
             const uint32_t sk = wbase_s + stage * Cfg::kStage;
+            // read once: first out of L2, so that a concurrent prefill keeps its re-read K/V tiles there
+            const uint64_t pol = l2_policy_evict_first();
             if (p.nhd) {
 #pragma unroll
                 for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-                    tma_load_3d(sk + hf * Cfg::kBox, &tm_k, hf * 64, h, y, bar);
-                    tma_load_3d(sk + Cfg::kTile + hf * Cfg::kBox, &tm_v, hf * 64, h, y, bar);
+                    tma_load_3d_hint(sk + hf * Cfg::kBox, &tm_k, hf * 64, h, y, bar, pol);
+                    tma_load_3d_hint(sk + Cfg::kTile + hf * Cfg::kBox, &tm_v, hf * 64, h, y, bar, pol);
                 }
             } else {
 #pragma unroll
                 for (int hf = 0; hf < Cfg::kHalves; ++hf) {
-                    tma_load_2d(sk + hf * Cfg::kBox, &tm_k, hf * 64, y, bar);
-                    tma_load_2d(sk + Cfg::kTile + hf * Cfg::kBox, &tm_v, hf * 64, y, bar);
+                    tma_load_2d_hint(sk + hf * Cfg::kBox, &tm_k, hf * 64, y, bar, pol);
+                    tma_load_2d_hint(sk + Cfg::kTile + hf * Cfg::kBox, &tm_v, hf * 64, y, bar, pol);
                 }
             }
         }

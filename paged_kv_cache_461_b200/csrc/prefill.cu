@@ -328,12 +328,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 }
                 if (lane == 0) {
                     const int ntiles = g.t1.rows ? 2 : 1;
+                    const uint64_t pol = l2_policy_evict_first(); // each Q row is read by one item only
                     mbar_arrive_expect_tx(bar + B_Q * 8, ntiles * Cfg::kTile);
                     for (int x = 0; x < ntiles; ++x)
 #pragma unroll
                         for (int hf = 0; hf < Cfg::kHalves; ++hf)
-                            tma_load_3d(sQ + x * Cfg::kTile + hf * Cfg::kHalfBytes, &tm_q, hf * 64, g.h * G,
-                                        g.qs + g.tok0 + x * TQ, bar + B_Q * 8);
+                            tma_load_3d_hint(sQ + x * Cfg::kTile + hf * Cfg::kHalfBytes, &tm_q, hf * 64, g.h * G,
+                                             g.qs + g.tok0 + x * TQ, bar + B_Q * 8, pol);
                 }
                 ++nq;
                 const int32_t *bt_row = p.bt + (int64_t)g.r * p.bt_stride;
