@@ -909,7 +909,7 @@ def main():
     ms_total = _time_region(st.step, args.steps, args.warmup, ws, window=win)
     # dominant kernel roofline: the attention launches (plan + decode with its split merge), events on their
     # stream, right after the timed steps (before the long window below warms the GPU into its power cap)
-    att_steps = max(20, min(args.steps, 200))
+    att_steps = max(50, min(args.steps, 200))
     att_ms = _attention_only_ms(st, att_steps)
     # the same step back to back for about 0.3 s, each step on its own events: the median per-step time, and
     # enough clock samples to see the clocks the timed steps ran at

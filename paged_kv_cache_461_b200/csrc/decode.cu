@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_kernel(const __grid_con
 
     const int u = (int)(blockIdx.x / (unsigned)p.Hkv);
     const int h = (int)(blockIdx.x % (unsigned)p.Hkv);
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+        p.hdr->write_epoch = kWriteEpochIdle; // the step's write launch (if any) has finished
     if (u >= (int)p.hdr->n_dec_units || (p.hdr->status & PA_DEVICE_WAIT_TIMEOUT))
         return; // past the work list, or an earlier CTA of this call already gave up
 

@@ -25,9 +25,15 @@ struct WsHeader {
     uint32_t n_reduce;    // decode requests with more than one split (merged by their last split CTA)
     uint32_t pf_ctas;     // persistent prefill CTAs that take work; the others leave their SM to decode
     uint32_t split_tokens; // keys per split-KV partition of this step's decode requests
-    uint32_t write_epoch;  // call id published once the status word is cleared (write-and-plan launch)
+    uint32_t write_epoch;  // call id published once the status word is cleared (write-and-plan launch);
+                           // kWriteEpochIdle once the step's attention kernels have started
     uint32_t pad[57];
 };
+
+// write_epoch between calls: the attention kernels of a step (which start only after its write-and-plan
+// launch has finished) set it to this value, which no call id takes.  A launch replayed from a CUDA graph
+// keeps its call id, so without the reset its writers could take the previous replay's epoch for this one's.
+constexpr uint32_t kWriteEpochIdle = 0xFFFFFFFFu;
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 // How a call is decomposed (host side, from the host hints only).

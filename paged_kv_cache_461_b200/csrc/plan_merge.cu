@@ -311,7 +311,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const AttnParams p, int n_bu
 // One launch for the start of a step: CTA 0 plans the step's attention while the other CTAs write its new
 // K/V rows into the cache (neither reads what the other writes).  A slot outside the pool sets
 // PA_DEVICE_BAD_SLOT in the status word, which CTA 0 clears for this call first: a writer that meets one
-// waits (bounded) until CTA 0 has published this call's epoch after the clear.
+// waits (bounded) until CTA 0 has published this call's epoch after the clear.  The step's attention
+// kernels set the epoch word back to kWriteEpochIdle, so the same launch replayed from a CUDA graph (same
+// epoch argument) waits for its own CTA 0 as well.
 template <int VEC>
 __global__ void __launch_bounds__(256) write_plan_kernel(const AttnParams p, int n_buckets, const KvWriteArgs w,
                                                          uint32_t epoch)
@@ -378,7 +380,9 @@ cudaError_t launch_write_plan(const AttnParams &p, const KvWriteArgs &w, bool ve
         n_buckets = 12 * 1024;
     const int smem = n_buckets * (int)sizeof(int);
     static std::atomic<uint32_t> epoch_counter{0};
-    const uint32_t epoch = ++epoch_counter;
+    uint32_t epoch = ++epoch_counter;
+    if (epoch == kWriteEpochIdle)
+        epoch = ++epoch_counter;
     const unsigned grid = 1u + (unsigned)kv_write_ctas(w.num_tokens);
     if (vec_ok)
         write_plan_kernel<8><<<grid, 256, smem, s>>>(p, n_buckets, w, epoch);

@@ -247,6 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                                                               const AttnParams p)
 {
     using Cfg = PfCfg<D>;
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+        p.hdr->write_epoch = kWriteEpochIdle; // the step's write launch (if any) has finished
     const int n_items = (int)p.hdr->n_pf_tiles * p.Hkv;
     // CTAs that take work: the plan's share of the SMs for prefill (the rest go to decode)
     const int n_ctas = min(min((int)gridDim.x, n_items), max(1, (int)p.hdr->pf_ctas));

@@ -327,6 +327,46 @@ def test_step_replays_from_a_cuda_graph_bit_identically(kind):
     assert api.read_device_status(st.workspace) == 0
 
 
+@pytest.mark.parametrize("bad_slot", [False, True])
+def test_mixed_write_replays_from_a_cuda_graph(bad_slot):
+    # the write-and-plan launch keeps its call id in a graph: every replay must still clear the status word
+    # before its writers report a slot outside the pool, and replay to the eager call's bits
+    rng = np.random.default_rng(43)
+    ctx = list(rng.integers(0, 2000, size=24)) + [0, 900]
+    q = [1] * 24 + [260, 97]
+    lay = _layout("graphw", ctx, q, 32, 8, 128, seed=23)
+    vals = W.make_values_numpy(lay, sentinel="pattern")
+    st = DevStep(lay, vals)
+    slots = lay.slot_mapping.copy()
+    if bad_slot:
+        slots[3] = lay.num_blocks * 16 + 7                # a decode token's slot outside the pool
+        slots[30] = lay.num_blocks * 16 + 100             # and a prefill token's
+    st.slots = torch.from_numpy(slots).cuda()
+    want = api.DEVICE_BAD_SLOT if bad_slot else 0
+    cap = torch.cuda.Stream()
+    with torch.cuda.stream(cap):                     # eager call on the capture stream first (side stream)
+        out_e, lse_e = write_and_attend_mixed(st)
+    torch.cuda.synchronize()
+    assert api.read_device_status(st.workspace) == want
+    out_g = torch.full_like(out_e, float("nan"))
+    lse_g = torch.full_like(lse_e, float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        api.attention_mixed_write(st.q, st.k_new, st.v_new, st.slots, st.k_cache, st.v_cache, st.qsl,
+                                  st.seq_lens, st.bt, lay.max_query_len, lay.max_seq_len, out=out_g, lse=lse_g,
+                                  workspace=st.workspace)
+    for _ in range(4):
+        st.workspace[:4].fill_(0xA5)                 # a stale status word: each replay clears it first
+        g.replay()
+        torch.cuda.synchronize()
+        assert api.read_device_status(st.workspace) == want
+        assert _bits_equal(out_g, out_e) and torch.equal(lse_g, lse_e)
+    written = np.where(slots < lay.num_blocks * 16, slots, -1)  # a slot outside the pool writes nothing
+    kc, vc = oracle.kv_write(vals.k_new, vals.v_new, written, vals.k_cache, vals.v_cache)
+    assert np.array_equal(to_host_bits(st.k_cache), kc)
+    assert np.array_equal(to_host_bits(st.v_cache), vc)
+
+
 @pytest.mark.parametrize("mode", ["fused_decode", "prefill_only"])
 def test_other_entry_points_replay_from_a_cuda_graph(mode):
     rng = np.random.default_rng(41)
