@@ -84,6 +84,7 @@ __device__ __forceinline__ void cta_excl_scan3(int a, int b, int c, int &ea, int
 // two rates balance.)
 constexpr float kPfFlopsPerSm = 6.2e12f;
 constexpr int kDecCtasPerSm = 12; // decode CTAs per SM below which the plan keeps the shorter split
+constexpr int kDecBuckets = 257;  // decode unit lengths in 128-key buckets (longer units share the last)
 constexpr float kDecBytesPerSm = 80e9f;
 constexpr float kDecBytesMax = 6.35e12f;
 
@@ -218,28 +219,64 @@ __device__ __forceinline__ void plan_body(const AttnParams &p, int n_buckets, in
         else if ((int64_t)carry_u2 * p.Hkv >= want)
             split = s2;
     }
-    // pass 1b: decode units in request order at that split size, split-arrival counters zeroed
+    // pass 1b: decode units at that split size, longest first: a counting sort over their key counts in
+    // 128-key buckets, so that the CTAs of the longest units start first and the grid ends on short ones
+    // (the decode grid is ragged: request lengths differ by up to 8x in one batch).  Split-arrival
+    // counters zeroed.
+    __shared__ int dec_hist[kDecBuckets];
+    for (int i = threadIdx.x; i < kDecBuckets; i += blockDim.x)
+        dec_hist[i] = 0;
+    __syncthreads();
+    auto dec_keys = [&](int r) { // keys of request r if it takes the decode kernel, else 0
+        if (p.num_seqs <= (int)blockDim.x)
+            return kept_L;
+        int n_dec, n_pf, red, ctx, q_len;
+        classify(r, n_dec, n_pf, red, ctx, q_len);
+        return n_dec ? ctx + q_len : 0;
+    };
+    auto dec_bucket = [&](int L, int u) {
+        const int len = min(split, L - u * split);
+        return min((len + 127) >> 7, kDecBuckets - 1);
+    };
     int carry_dec = 0, carry_red = 0;
     for (int base = 0; base < p.num_seqs; base += blockDim.x) {
         const int r = base + threadIdx.x;
-        int L = kept_L;
-        if (p.num_seqs > (int)blockDim.x) {
-            int n_dec, n_pf, red, ctx, q_len;
-            classify(r, n_dec, n_pf, red, ctx, q_len);
-            L = n_dec ? ctx + q_len : 0;
-        }
+        const int L = dec_keys(r);
         const int n_dec = (L + split - 1) / split;
         const int red = n_dec > 1 ? 1 : 0;
         int ed, er, e2, td, tr, t2;
         cta_excl_scan3(n_dec, red, 0, ed, er, e2, td, tr, t2);
         for (int u = 0; u < n_dec; ++u)
-            if (carry_dec + ed + u < p.max_dec_units)
-                p.dec_units[carry_dec + ed + u] = make_int2(r, u);
+            atomicAdd(&dec_hist[dec_bucket(L, u)], 1);
         if (red)
             for (int h = 0; h < p.Hkv; ++h)
                 p.split_arrivals[(int64_t)r * p.Hkv + h] = 0u; // counted by the decode kernel
         carry_dec += td;
         carry_red += tr;
+    }
+    __syncthreads();
+    {
+        int carry = 0; // bucket start offsets, longest bucket first
+        for (int base = 0; base < kDecBuckets; base += blockDim.x) {
+            const int b = kDecBuckets - 1 - (base + (int)threadIdx.x);
+            const int cnt = b >= 0 ? dec_hist[b] : 0;
+            int e0, e1, e2, t0, t1, t2;
+            cta_excl_scan3(cnt, 0, 0, e0, e1, e2, t0, t1, t2);
+            if (b >= 0)
+                dec_hist[b] = carry + e0;
+            carry += t0;
+            __syncthreads();
+        }
+    }
+    for (int base = 0; base < p.num_seqs; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        const int L = dec_keys(r);
+        const int n_dec = (L + split - 1) / split;
+        for (int u = 0; u < n_dec; ++u) {
+            const int pos = atomicAdd(&dec_hist[dec_bucket(L, u)], 1);
+            if (pos < p.max_dec_units)
+                p.dec_units[pos] = make_int2(r, u);
+        }
     }
     __syncthreads();
     if (carry_pf > 0) { // a step without prefill work skips the sort
