@@ -134,7 +134,7 @@ __device__ __forceinline__ int pair_cost(int ctx, int q_len, int qp, int tq)
     return (ctx + last) / 128 + 1;
 }
 
-// Work lists of one step.  Decode units in request order; prefill q-pairs sorted by
+// Work lists of one step.  Decode units longest first (see pass 1b); prefill q-pairs sorted by
 // cost (key steps), most expensive first -- a counting sort through a shared-memory
 // histogram, so the persistent prefill CTAs, which walk the list in snake order, end
 // at nearly the same time.  Pairs of equal cost land in any order; every pair is
