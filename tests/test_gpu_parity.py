@@ -491,6 +491,30 @@ def test_plan_picks_the_split_size_per_step(n_req, lo, hi, n_pf):
         assert st.workspace[20:24].view(torch.int32).item() == 1024
 
 
+@pytest.mark.parametrize("with_prefill", [False, True])
+def test_plan_lists_decode_units_longest_first(with_prefill):
+    # the plan lists every decode unit (request, split index) once, longest first in 128-key buckets, so that
+    # the ragged decode grid ends on short CTAs; a prefill chunk in the step does not enter the list
+    rng = np.random.default_rng(61 + int(with_prefill))
+    ctx = list(rng.integers(1, 5000, size=57)) + ([700] if with_prefill else [])
+    q = [1] * 57 + ([200] if with_prefill else [])
+    lay = _layout("unitorder", ctx, q, 32, 8, 128, seed=61)
+    st = DevStep(lay, W.make_values_numpy(lay))
+    st.write()
+    st.attend()
+    torch.cuda.synchronize()
+    assert api.read_device_status(st.workspace) == 0
+    hdr = st.workspace[:64].view(torch.int32).cpu().tolist()
+    n_dec, s = hdr[1], hdr[5]
+    units = st.workspace[256:256 + 8 * n_dec].view(torch.int32).cpu().numpy().reshape(-1, 2)
+    L = lay.seq_lens
+    want = sorted((r, u) for r in range(57) for u in range((int(L[r]) + s - 1) // s))
+    assert sorted(map(tuple, units.tolist())) == want
+    lens = np.minimum(s, L[units[:, 0]] - units[:, 1] * s)
+    buckets = (lens + 127) // 128
+    assert np.all(np.diff(buckets) <= 0), "decode units not longest first"
+
+
 # ----------------------------------------------------------------------------- device-side checks
 
 def test_bad_metadata_sets_status_and_never_faults():
